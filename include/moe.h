@@ -1,0 +1,260 @@
+/* split_weight_b200: the data-parallel MoE expert block of DWDP on one B200.
+ *
+ * DWDP ("DWDP: Distributed Weight Data Parallelism for High-Performance LLM
+ * Inference on NVL72", arXiv 2604.01621, abstract) keeps every GPU data
+ * parallel: a rank runs the MoE block on its own tokens, and only the expert
+ * weights are split between peers, the missing ones being fetched
+ * asynchronously instead of through a layer-boundary collective.  The
+ * explainer "Distributed Weight Data Parallelism cuts LLM inference stalls"
+ * shows (split-weight figure) that the local and remote expert weights have
+ * to reach the grouped GEMM; this library reaches them through a per-expert
+ * (pool, slot) table spanning both pools, with no merge copy, and prefetches
+ * the next layer's remote experts into an alternate buffer on a copy-engine
+ * stream (prefetch-timeline figure).
+ *
+ * One layer, all calls enqueued on one compute stream:
+ *   moe_route -> moe_permute -> moe_grouped_ffn -> moe_combine
+ * and, on a copy stream, moe_prefetch_layer for a later layer.
+ *
+ * Conventions (all entry points):
+ *   - Every function returns a moe_status; nothing aborts, exits or traps.
+ *     moe_last_error() gives a thread-local description of the last failure.
+ *   - Shapes, pointers and alignment are checked on the host before any
+ *     launch; a bad argument returns MOE_ERR_INVALID_ARG (or
+ *     MOE_ERR_UNSUPPORTED for a legal but unimplemented case) and enqueues
+ *     nothing.
+ *   - The caller owns all memory.  The library allocates no device memory;
+ *     calls that need scratch take (workspace, workspace_bytes), sized by the
+ *     matching *_workspace_size query; too small -> MOE_ERR_WORKSPACE.
+ *   - Device pointers must be 16-byte aligned.  Every call is asynchronous on
+ *     the given stream and never synchronises.  Errors of the launch itself
+ *     return MOE_ERR_CUDA; faults inside a kernel surface at the caller's
+ *     next synchronisation.  Kernels never wait without a time limit: a wait
+ *     that runs out sets the device error word that moe_check_device() reads
+ *     (MOE_ERR_TIMEOUT) and the kernel returns.
+ *   - Matrices are row-major.  bf16 is IEEE bfloat16, e4m3 is the OCP FP8
+ *     E4M3 "fn" format (max 448, no infinities).
+ */
+#ifndef SPLIT_WEIGHT_B200_MOE_H
+#define SPLIT_WEIGHT_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOPK 32
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_WORKSPACE = 3,
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_TIMEOUT = 5,
+    MOE_ERR_DEVICE_CHECK = 6
+} moe_status;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
+
+typedef enum moe_score { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+
+/* Static text for a status code. */
+MOE_API const char *moe_status_string(moe_status s);
+/* Thread-local description of the last failing call ("" if none). */
+MOE_API const char *moe_last_error(void);
+/* MOE_ABI_VERSION of the loaded library. */
+MOE_API int32_t moe_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Routing: router logits, scores and top-k selection.
+ *
+ * The pages run "the MoE expert layer" of DeepSeek-R1 on every rank (arXiv
+ * 2604.01621, abstract; explainer, first figure) but give no router
+ * arithmetic; this is the DeepSeek-R1 layer shape read plainly:
+ *   logits  l[t,e] = sum_h x[t,h] W_g[e,h] in fp32, in a fixed order: h in
+ *           chunks of 256, each a chain of fused multiply-adds from 0 in
+ *           ascending h, the chunk sums added in ascending order.
+ *   SOFTMAX: the k largest logits; w_j = exp(l_j - l_max) / sum over the k
+ *           chosen (renormalize != 0) or over all E (renormalize == 0).
+ *   SIGMOID: s = sigmoid(l) (evaluated in fp64, rounded to fp32); selection
+ *           key s + bias[e] (fp32); groups are n_group contiguous blocks of
+ *           E/n_group experts scored by the sum of their two largest keys;
+ *           the topk_group best groups are kept and the k best keys inside
+ *           them chosen; w_j = s_j / sum_i s_i (fp32, i in output order) when
+ *           renormalize != 0, else s_j.
+ *   Both: w_j *= routed_scale.  Ties go to the lower index everywhere.
+ * Results are bit-for-bit reproducible (the exponent of the sigmoid is this
+ * library's own fp64 routine).
+ *
+ * x        [T, H] device, dtype MOE_F32 or MOE_BF16.
+ * w_gate   [E, H] fp32 device.   bias [E] fp32 device or NULL (SIGMOID only).
+ * topk_idx [T, k] int32 out, experts in descending key order.
+ * topk_w   [T, k] fp32 out.
+ * Limits: 1 <= E <= 1024, 1 <= k <= 32, H % 32 == 0, T >= 0;
+ *         SIGMOID: E % n_group == 0, n_group <= 32,
+ *                  1 <= topk_group <= n_group, k <= topk_group * E / n_group.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_route_cfg {
+    int32_t T, H, E, k;
+    int32_t score;       /* moe_score */
+    int32_t n_group;     /* SIGMOID: number of expert groups (1 = no grouping) */
+    int32_t topk_group;  /* SIGMOID: groups kept per token */
+    float routed_scale;  /* multiplies every routing weight */
+    int32_t renormalize; /* see above */
+} moe_route_cfg;
+
+MOE_API size_t moe_route_workspace_size(const moe_route_cfg *cfg);
+MOE_API moe_status moe_route(const moe_route_cfg *cfg, const void *x, moe_dtype x_dtype,
+                     const float *w_gate, const float *bias, int32_t *topk_idx, float *topk_w,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Permutation: expert histogram, scan, stable scatter and row gather.
+ *
+ * Groups each rank's token-expert assignments by expert so that one grouped
+ * GEMM serves all of them (explainer, split-weight figure: the grouped GEMM
+ * of the block).  With a = t*k + j the assignments in ascending order:
+ *   offsets[e]  = number of assignments to experts < e   ([E+1], offsets[E] = T*k)
+ *   row of a    = offsets[e] + #{a' < a with the same expert}   (stable)
+ *   perm_src[row] = t,  inv_pos[t,j] = row
+ *   x_perm[row]   = x[t] converted to perm_dtype;
+ *   with_shared != 0: rows T*k .. T*k+T-1 of x_perm are x[0..T-1] (input of
+ *   the always-on shared expert).
+ * perm_dtype MOE_BF16: x_perm [rows, H] bf16 (fp32 x is rounded to nearest
+ * even).  perm_dtype MOE_E4M3: x_perm [rows, H] e4m3 plus x_perm_scales
+ * [rows, H/128] fp32, per 128 columns s = amax/448, code = e4m3(v/s).
+ * topk_idx entries must lie in [0, E) (checked on the device: an entry
+ * outside sets the device error word, MOE_ERR_DEVICE_CHECK, and is skipped).
+ * Limits: H % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.
+ * ---------------------------------------------------------------------- */
+MOE_API size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
+MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t *topk_idx,
+                       const void *x, moe_dtype x_dtype, moe_dtype perm_dtype, int32_t with_shared,
+                       int32_t *offsets, int32_t *perm_src, int32_t *inv_pos, void *x_perm,
+                       float *x_perm_scales, void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Expert weight images and the split-weight table.
+ *
+ * One expert image (a "slot") holds, at the offsets moe_expert_layout_get
+ * returns: w_gu [2I, H] (gate rows 0..I-1, up rows I..2I-1) and w_down
+ * [H, I], both row-major in w_dtype; for MOE_E4M3 also fp32 block scales
+ * s_gu [2I/128, H/128] and s_down [H/128, I/128] (weight = code * scale).
+ * A pool is `count` slots `stride` bytes apart (stride >= layout.bytes,
+ * stride % 256 == 0, base 1024-byte aligned).
+ *
+ * The table spans two pools that need not be adjacent or related in any way
+ * (the explainer's split-weight figure: local and remote weights reach the
+ * grouped GEMM without being merged into one contiguous buffer):
+ *   pool_slot[e] = (pool << 31) | slot,  pool 0 = local, pool 1 = remote.
+ * pool_slot is a HOST array of E entries, read during the call.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_expert_layout {
+    int64_t gu_offset, down_offset;             /* bytes from the slot start */
+    int64_t gu_scale_offset, down_scale_offset; /* -1 unless MOE_E4M3 */
+    int64_t bytes;                              /* bytes of one image (256-byte multiple) */
+} moe_expert_layout;
+
+MOE_API moe_status moe_expert_layout_get(int32_t H, int32_t I, moe_dtype w_dtype, moe_expert_layout *out);
+
+typedef struct moe_expert_table {
+    const void *local_base;
+    int32_t local_count;
+    int64_t local_stride;
+    const void *remote_base;
+    int32_t remote_count;
+    int64_t remote_stride;
+    const void *shared;        /* one image of the shared expert, or NULL */
+    const int32_t *pool_slot;  /* HOST [E] */
+} moe_expert_table;
+
+/* ------------------------------------------------------------------------
+ * Grouped SwiGLU expert FFN over the split pools (the block's grouped GEMM;
+ * explainer, split-weight figure).
+ *
+ * For every routed expert e with n_e = offsets[e+1] - offsets[e] > 0 and,
+ * when has_shared, for the shared expert on rows T*k .. T*k+T-1:
+ *   G = X_e W_gu[e]^T                     X_e = x_perm rows of e
+ *   h = silu(G[:, :I]) * G[:, I:]         -> h rows of e   (bf16)
+ *   y = h W_down[e]^T                     -> y_perm rows of e (bf16)
+ * fp32 accumulation on the tensor cores.
+ * x_perm  [rows, H] act_dtype (rows = T*k + (has_shared ? T : 0)).
+ * h       [rows, I] bf16 (intermediate, caller-owned).
+ * y_perm  [rows, H] bf16 out.
+ * Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024; w_dtype MOE_BF16 with
+ * act_dtype MOE_BF16, or w_dtype MOE_E4M3 with act_dtype MOE_BF16.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_ffn_desc {
+    int32_t T, H, I, E, k;
+    int32_t w_dtype;    /* moe_dtype of the expert weights */
+    int32_t act_dtype;  /* moe_dtype of x_perm */
+    int32_t has_shared; /* shared expert present */
+} moe_ffn_desc;
+
+MOE_API size_t moe_grouped_ffn_workspace_size(const moe_ffn_desc *d);
+MOE_API moe_status moe_grouped_ffn(const moe_ffn_desc *d, const moe_expert_table *tbl, const void *x_perm,
+                           const float *x_perm_scales, const int32_t *offsets, void *h,
+                           void *y_perm, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Weighted combine (unpermute):
+ *   y[t] = sum_{j=0..k-1, ascending} topk_w[t,j] * y_perm[inv_pos[t,j]]
+ *          + (with_shared ? y_perm[T*k + t] : 0)
+ * in fp32, rounded once to y_dtype (MOE_F32 or MOE_BF16).
+ * y_perm [rows, H] bf16; inv_pos [T, k] int32; topk_w [T, k] fp32; y [T, H].
+ * Limits: H % 8 == 0, 1 <= k <= 32.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_combine(int32_t T, int32_t k, int32_t H, const void *y_perm, const int32_t *inv_pos,
+                       const float *topk_w, int32_t with_shared, void *y, moe_dtype y_dtype,
+                       cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Remote-expert prefetch into the alternate buffer (explainer, prefetch
+ * figure: while a rank computes layer l, the copy engine fetches layer l+1's
+ * remote experts into the alternate buffer; fetch-path figure: the pull is a
+ * cudaMemcpyAsync on the copy engine, not on the SMs).
+ *
+ * Enqueues on copy_stream: a wait on wait_free (if not NULL: the event the
+ * compute stream recorded after the last use of dst), the copy of `bytes`
+ * from src to dst (cudaMemcpyAsync device-to-device, in pieces of
+ * chunk_bytes if chunk_bytes > 0), and a record of ready_out (if not NULL),
+ * which the consumer waits on before moe_grouped_ffn reads dst.  src may be
+ * another GPU's memory when peer access is enabled.
+ * ---------------------------------------------------------------------- */
+MOE_API moe_status moe_prefetch_layer(const void *src, void *dst, size_t bytes, size_t chunk_bytes,
+                              cudaStream_t copy_stream, cudaEvent_t wait_free,
+                              cudaEvent_t ready_out);
+
+/* Host-side poll of an event with a deadline: MOE_OK once it has completed,
+ * MOE_ERR_TIMEOUT after timeout_ms milliseconds, MOE_ERR_CUDA on error. */
+MOE_API moe_status moe_wait_ready(cudaEvent_t ev, int32_t timeout_ms);
+
+/* Synchronises the current device, then reads and clears the device error
+ * word: MOE_OK, MOE_ERR_TIMEOUT (a kernel wait ran out) or
+ * MOE_ERR_DEVICE_CHECK (an index outside its range was seen and skipped). */
+MOE_API moe_status moe_check_device(void);
+
+/* Test hook: the next `count` CUDA runtime calls the library makes report
+ * failure (MOE_ERR_CUDA) without being issued.  0 disarms it. */
+MOE_API void moe_debug_fail_next_cuda_calls(int32_t count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPLIT_WEIGHT_B200_MOE_H */

@@ -1,0 +1,218 @@
+// Library-wide entry points: status text, errors, the device error word,
+// tensor-map encoding, expert image layout and the copy-engine prefetch.
+#include <atomic>
+#include <chrono>
+#include <cstring>
+#include <mutex>
+#include <thread>
+
+#include "internal.h"
+
+namespace swb {
+
+namespace {
+thread_local char g_last_error[512] = "";
+std::atomic<int> g_fail_next{0};
+
+// One error word per device, in device memory owned by this library's
+// module (a __device__ variable: the library still allocates nothing).
+__device__ int g_device_error_word;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {0};
+int* g_err_word[kMaxDevices] = {nullptr};
+}  // namespace
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+bool cuda_injected_failure() {
+    int n = g_fail_next.load();
+    while (n > 0) {
+        if (g_fail_next.compare_exchange_weak(n, n - 1)) return true;
+    }
+    return false;
+}
+
+moe_status cuda_check(cudaError_t e, const char* what) {
+    return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+moe_status device_error_word(int** out) {
+    int dev = 0;
+    SWB_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_err_word[dev]) {
+        void* p = nullptr;
+        SWB_CUDA(cudaGetSymbolAddress(&p, g_device_error_word));
+        g_err_word[dev] = static_cast<int*>(p);
+    }
+    *out = g_err_word[dev];
+    return MOE_OK;
+}
+
+moe_status sm_count(int* out) {
+    int dev = 0;
+    SWB_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device %d", dev);
+    if (!g_sm_count[dev]) {
+        int n = 0;
+        SWB_CUDA(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev));
+        g_sm_count[dev] = n;
+    }
+    *out = g_sm_count[dev];
+    return MOE_OK;
+}
+
+moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, void* base,
+                        const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                        CUtensorMapSwizzle swizzle) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cuda_injected_failure())
+                return fail(MOE_ERR_CUDA, "cudaGetDriverEntryPoint: injected failure");
+            cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn,
+                                                    cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+    }
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5], es[5];
+    for (uint32_t i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) s[i] = strides_bytes[i];
+    }
+    CUresult r = g_encode(map, dtype, rank, base, d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MOE_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return MOE_OK;
+}
+
+}  // namespace swb
+
+using namespace swb;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+        case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_error(void) { return g_last_error; }
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+void moe_debug_fail_next_cuda_calls(int32_t count) { g_fail_next.store(count > 0 ? count : 0); }
+
+moe_status moe_expert_layout_get(int32_t H, int32_t I, moe_dtype w_dtype, moe_expert_layout* out) {
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "moe_expert_layout_get: out is NULL");
+    if (H <= 0 || I <= 0 || H % 128 || I % 128)
+        return fail(MOE_ERR_INVALID_ARG, "moe_expert_layout_get: H=%d I=%d must be positive "
+                    "multiples of 128", H, I);
+    auto up = [](int64_t v) { return (v + 255) / 256 * 256; };
+    int64_t es;
+    if (w_dtype == MOE_BF16) es = 2;
+    else if (w_dtype == MOE_E4M3) es = 1;
+    else return fail(MOE_ERR_UNSUPPORTED, "moe_expert_layout_get: weight dtype %d", (int)w_dtype);
+    const int64_t gu = 2LL * I * H * es, dn = (int64_t)H * I * es;
+    out->gu_offset = 0;
+    out->down_offset = up(gu);
+    int64_t end = out->down_offset + up(dn);
+    out->gu_scale_offset = out->down_scale_offset = -1;
+    if (w_dtype == MOE_E4M3) {
+        out->gu_scale_offset = end;
+        end += up((2LL * I / 128) * (H / 128) * 4);
+        out->down_scale_offset = end;
+        end += up((int64_t)(H / 128) * (I / 128) * 4);
+    }
+    out->bytes = end;
+    return MOE_OK;
+}
+
+moe_status moe_prefetch_layer(const void* src, void* dst, size_t bytes, size_t chunk_bytes,
+                              cudaStream_t copy_stream, cudaEvent_t wait_free,
+                              cudaEvent_t ready_out) {
+    if (bytes > 0 && (!src || !dst))
+        return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer: NULL buffer");
+    if (bytes > 0) {
+        const char* s = static_cast<const char*>(src);
+        char* d = static_cast<char*>(dst);
+        if ((s < d + bytes) && (d < s + bytes))
+            return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer: source and destination overlap");
+    }
+    if (wait_free) SWB_CUDA(cudaStreamWaitEvent(copy_stream, wait_free, 0));
+    size_t step = chunk_bytes ? chunk_bytes : bytes;
+    for (size_t off = 0; off < bytes; off += step) {
+        size_t n = bytes - off < step ? bytes - off : step;
+        SWB_CUDA(cudaMemcpyAsync(static_cast<char*>(dst) + off,
+                                 static_cast<const char*>(src) + off, n,
+                                 cudaMemcpyDeviceToDevice, copy_stream));
+    }
+    if (ready_out) SWB_CUDA(cudaEventRecord(ready_out, copy_stream));
+    return MOE_OK;
+}
+
+moe_status moe_wait_ready(cudaEvent_t ev, int32_t timeout_ms) {
+    if (!ev) return fail(MOE_ERR_INVALID_ARG, "moe_wait_ready: NULL event");
+    const auto t0 = std::chrono::steady_clock::now();
+    while (true) {
+        if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "cudaEventQuery: injected failure");
+        cudaError_t e = cudaEventQuery(ev);
+        if (e == cudaSuccess) return MOE_OK;
+        if (e != cudaErrorNotReady) return cuda_check(e, "cudaEventQuery");
+        auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(
+                      std::chrono::steady_clock::now() - t0).count();
+        if (ms >= timeout_ms)
+            return fail(MOE_ERR_TIMEOUT, "moe_wait_ready: event not complete after %d ms",
+                        (int)timeout_ms);
+        std::this_thread::sleep_for(std::chrono::microseconds(100));
+    }
+}
+
+moe_status moe_check_device(void) {
+    int* w = nullptr;
+    moe_status st = device_error_word(&w);
+    if (st != MOE_OK) return st;
+    SWB_CUDA(cudaDeviceSynchronize());
+    int v = 0;
+    SWB_CUDA(cudaMemcpy(&v, w, sizeof v, cudaMemcpyDeviceToHost));
+    if (v) {
+        int zero = 0;
+        SWB_CUDA(cudaMemcpy(w, &zero, sizeof zero, cudaMemcpyHostToDevice));
+        if (v & kDevErrTimeout) return fail(MOE_ERR_TIMEOUT, "a kernel wait ran out (word %d)", v);
+        return fail(MOE_ERR_DEVICE_CHECK, "device check failed (word %d)", v);
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,474 @@
+// moe_grouped_ffn: grouped SwiGLU expert GEMMs over split weight pools.
+//
+// The block's grouped GEMM (explainer "Distributed Weight Data Parallelism
+// cuts LLM inference stalls", split-weight figure) must read each expert's
+// weights wherever they sit: in this rank's local pool or in the buffer the
+// remote experts were fetched into.  Instead of merging the two into one
+// contiguous buffer, every pool gets a 3-D TMA tensor map {K, rows, slot};
+// an expert is (pool, slot) in the per-expert table, so the producer warp
+// simply picks the map and passes the slot as the third coordinate.
+//
+// One persistent, warp-specialised kernel per GEMM (sm_100a):
+//   warp 0      TMA producer (one thread): weight tile(s) + token rows
+//   warp 1      tcgen05.mma issuer (one thread); owns the TMEM allocation
+//   warps 2-5   epilogue: TMEM -> registers -> (SwiGLU) -> bf16 -> global
+// The MMA puts the weight rows on M (128) and the expert's tokens on N
+// (16..BN), so a decode-sized expert with 4 tokens costs an N=16 MMA, not a
+// 128-row tile.  GEMM1 keeps two fp32 accumulators per tile, gate and up for
+// the same 128 features, so SwiGLU is fused in the epilogue.  Accumulators
+// are double buffered in TMEM so the epilogue of one tile overlaps the next
+// tile's main loop.
+#include <cuda_bf16.h>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace swb {
+namespace {
+
+constexpr int kMaxGroups = MOE_MAX_EXPERTS + 1;
+constexpr int kBM = 128;                       // weight rows per tile (MMA M)
+constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle atom
+constexpr int kBoxN = 16;                      // token rows per TMA box
+constexpr uint32_t kABytes = kBM * kBK * 2;    // one weight tile, 16 KB
+constexpr int kThreads = 192;
+constexpr uint32_t kSmemBudget = 200 * 1024;   // pipeline stages
+
+struct alignas(64) FfnArgs {
+    CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}
+    CUtensorMap act_map;       // activation rows {K, rows}
+    const int32_t* offsets;    // [E+1] first row of each expert
+    __nv_bfloat16* out;        // [rows, ld_out]
+    int* err;                  // device error word
+    int32_t E, T, A, has_shared;
+    int32_t K;                 // reduction length (H for GEMM1, I for GEMM2)
+    int32_t M;                 // output features per expert (I for GEMM1, H for GEMM2)
+    int32_t up_row;            // GEMM1: first row of the "up" half of w_gu (= I)
+    int32_t ld_out;
+    int32_t pool_slot[kMaxGroups];  // (pool << 31) | slot per routed expert
+};
+
+template <int BN, bool GATED>
+struct Cfg {
+    static constexpr uint32_t kAStage = kABytes * (GATED ? 2 : 1);
+    static constexpr uint32_t kStageBytes = kAStage + BN * kBK * 2;
+    static constexpr int kStages = (kSmemBudget / kStageBytes) > 12 ? 12 : (kSmemBudget / kStageBytes);
+    static constexpr uint32_t kAccCols = (GATED ? 2 : 1) * BN;
+    static constexpr uint32_t kTmemCols = 2 * kAccCols;
+    static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024;
+};
+
+struct Tile {
+    int m0, row0, n_rows, n_mma, map, slot;
+};
+
+struct Tables {
+    int tile_start[kMaxGroups + 1];
+    int row0[kMaxGroups];
+    int n[kMaxGroups];
+    int ps[kMaxGroups];  // (map << 24) | slot   (map 0 local, 1 remote, 2 shared)
+};
+
+template <int BN>
+__device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G, int MT) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {  // largest group whose first tile is <= tile (never an empty one)
+        const int mid = (lo + hi + 1) >> 1;
+        if (tb.tile_start[mid] <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    const int g = lo, local = tile - tb.tile_start[g], n = tb.n[g];
+    const int ntn = (n + BN - 1) / BN;
+    const int mt = local / ntn, nt = local - mt * ntn;
+    Tile t;
+    t.m0 = mt * kBM;
+    t.row0 = tb.row0[g] + nt * BN;
+    t.n_rows = min(BN, n - nt * BN);
+    t.n_mma = (t.n_rows + 15) & ~15;
+    t.map = tb.ps[g] >> 24;
+    t.slot = tb.ps[g] & 0xFFFFFF;
+    (void)MT;
+    return t;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+template <int BN, bool GATED>
+__global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_constant__ FfnArgs p) {
+    using C = Cfg<BN, GATED>;
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ Tables tb;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t stages = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    const int G = p.E + (p.has_shared ? 1 : 0);
+    const int MT = p.M / kBM;
+    const int KB = p.K / kBK;
+    volatile int* abort_flag = &abort_sh;
+
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&acc_full[a]), 1);
+            mbar_init(smem_u32(&acc_empty[a]), 4);
+        }
+        fence_mbar_init();
+        tma_prefetch_map(&p.act_map);
+        for (int m = 0; m < 3; ++m) tma_prefetch_map(&p.w_map[m]);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 2) {
+        // per-group rows, tiles and (pool, slot); exclusive scan of tiles
+        const int per = (G + 31) / 32, g0 = lane * per, g1 = min(G, g0 + per);
+        int sum = 0;
+        for (int g = g0; g < g1; ++g) {
+            int n, r0, ps;
+            if (g < p.E) {
+                r0 = p.offsets[g];
+                n = p.offsets[g + 1] - r0;
+                const uint32_t v = static_cast<uint32_t>(p.pool_slot[g]);
+                ps = (int)(((v >> 31) << 24) | (v & 0xFFFFFFu));
+            } else {
+                r0 = p.A;
+                n = p.T;
+                ps = 2 << 24;
+            }
+            tb.row0[g] = r0;
+            tb.n[g] = n;
+            tb.ps[g] = ps;
+            sum += ((n + BN - 1) / BN) * MT;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int g = g0; g < g1; ++g) {
+            tb.tile_start[g] = run;
+            run += ((tb.n[g] + BN - 1) / BN) * MT;
+        }
+        if (lane == 31) tb.tile_start[G] = incl;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+    const int total = tb.tile_start[G];
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile<BN>(tile, tb, G, MT);
+                const CUtensorMap* wm = &p.w_map[t.map];
+                const uint32_t tx = C::kAStage + (uint32_t)t.n_mma * kBK * 2;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const uint32_t eb = smem_u32(&empty_bar[stage]);
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    if (!mbar_wait(eb, phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    mbar_arrive_expect_tx(fb, tx);
+                    tma_load_3d(sa, wm, fb, kb * kBK, t.m0, t.slot);
+                    if constexpr (GATED) tma_load_3d(sa + kABytes, wm, fb, kb * kBK, p.up_row + t.m0, t.slot);
+                    const uint32_t sb = sa + C::kAStage;
+                    for (int i = 0; i < t.n_mma / kBoxN; ++i)
+                        tma_load_2d(sb + i * kBoxN * kBK * 2, &p.act_map, fb, kb * kBK,
+                                    t.row0 + i * kBoxN);
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_use[2] = {0u, 0u};
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile<BN>(tile, tb, G, MT);
+                if (!mbar_wait(smem_u32(&acc_empty[acc]), (acc_use[acc] & 1u) ^ 1u, abort_flag,
+                               p.err))
+                    break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * C::kAccCols;
+                const uint32_t idesc = idesc_bf16_f32(kBM, t.n_mma);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    const uint32_t sb = sa + C::kAStage;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint32_t accum = (kb | kk) != 0;
+                        const uint64_t bd = sw128_desc(sb + kk * 32);
+                        mma_bf16_ss(d0, sw128_desc(sa + kk * 32), bd, idesc, accum);
+                        if constexpr (GATED)
+                            mma_bf16_ss(d0 + BN, sw128_desc(sa + kABytes + kk * 32), bd, idesc, accum);
+                    }
+                    mma_commit(smem_u32(&empty_bar[stage]));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&acc_full[acc]));
+                ++acc_use[acc];
+                acc ^= 1;
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int acc = 0;
+        uint32_t acc_use[2] = {0u, 0u};
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile<BN>(tile, tb, G, MT);
+            bool ok = mbar_wait(smem_u32(&acc_full[acc]), acc_use[acc] & 1u, abort_flag, p.err);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::kAccCols;
+            const int f = t.m0 + 32 * q + lane;
+            __nv_bfloat16* out = p.out + (int64_t)t.row0 * p.ld_out + f;
+            for (int c0 = 0; c0 < t.n_rows; c0 += 16) {
+                float g[16];
+                tmem_ld_16(tacc + c0, g);
+                if constexpr (GATED) {
+                    float u[16];
+                    tmem_ld_16(tacc + BN + c0, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.n_rows)
+                            out[(int64_t)(c0 + i) * p.ld_out] = __float2bfloat16_rn(silu_mul(g[i], u[i]));
+                } else {
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.n_rows)
+                            out[(int64_t)(c0 + i) * p.ld_out] = __float2bfloat16_rn(g[i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+            ++acc_use[acc];
+            acc ^= 1;
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {  // let copies still in flight land before TMEM is released
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+template <int BN, bool GATED>
+moe_status launch(const FfnArgs& a, int rows, int G, cudaStream_t s) {
+    using C = Cfg<BN, GATED>;
+    int sms = 0;
+    moe_status st = sm_count(&sms);
+    if (st != MOE_OK) return st;
+    const int64_t mt = a.M / kBM;
+    const int64_t bound = mt * ((rows + BN - 1) / BN + G);
+    const int grid = (int)(bound < sms ? bound : sms);
+    if (grid <= 0) return MOE_OK;
+    auto kern = k_grouped_ffn<BN, GATED>;
+    SWB_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)C::kDynSmem));
+    kern<<<grid, kThreads, C::kDynSmem, s>>>(a);
+    SWB_LAUNCHED(GATED ? "moe_grouped_ffn: gate/up kernel" : "moe_grouped_ffn: down kernel");
+    return MOE_OK;
+}
+
+template <bool GATED>
+moe_status launch_bn(int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) {
+    switch (bn) {
+        case 16: return launch<16, GATED>(a, rows, G, s);
+        case 32: return launch<32, GATED>(a, rows, G, s);
+        case 64: return launch<64, GATED>(a, rows, G, s);
+        default: return launch<128, GATED>(a, rows, G, s);
+    }
+}
+
+// Token tile: about twice the mean tokens per expert, 16..128.
+int pick_bn(int64_t A, int E) {
+    const int64_t mean = (A + E - 1) / E;
+    if (mean <= 8) return 16;
+    if (mean <= 16) return 32;
+    if (mean <= 32) return 64;
+    return 128;
+}
+
+moe_status encode_weight_map(CUtensorMap* m, const void* base, int64_t offset, int32_t count,
+                             int64_t stride, int32_t K, int32_t rows) {
+    const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)count};
+    const uint64_t strides[2] = {(uint64_t)K * 2, (uint64_t)stride};
+    const uint32_t box[3] = {(uint32_t)kBK, (uint32_t)kBM, 1u};
+    return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<char*>(static_cast<const char*>(base)) + offset, dims, strides,
+                        box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+moe_status encode_act_map(CUtensorMap* m, const void* base, int64_t rows, int32_t K) {
+    const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
+    const uint64_t strides[1] = {(uint64_t)K * 2};
+    const uint32_t box[2] = {(uint32_t)kBK, (uint32_t)kBoxN};
+    return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+moe_status validate(const moe_ffn_desc* d, const moe_expert_table* tb, moe_expert_layout* lay) {
+    if (!d || !tb) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: NULL descriptor or table");
+    if (d->T < 0 || d->k <= 0 || d->k > MOE_MAX_TOPK || d->E <= 0 || d->E > MOE_MAX_EXPERTS ||
+        d->H <= 0 || d->I <= 0 || d->H % 128 || d->I % 128)
+        return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: T=%d H=%d I=%d E=%d k=%d", d->T, d->H,
+                    d->I, d->E, d->k);
+    if (d->w_dtype != MOE_BF16 || d->act_dtype != MOE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "moe_grouped_ffn: weight dtype %d / activation dtype %d",
+                    d->w_dtype, d->act_dtype);
+    moe_status st = moe_expert_layout_get(d->H, d->I, (moe_dtype)d->w_dtype, lay);
+    if (st != MOE_OK) return st;
+    if (!tb->pool_slot) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: pool_slot is NULL");
+    const void* base[2] = {tb->local_base, tb->remote_base};
+    const int32_t count[2] = {tb->local_count, tb->remote_count};
+    const int64_t stride[2] = {tb->local_stride, tb->remote_stride};
+    for (int q = 0; q < 2; ++q) {
+        if (count[q] < 0 || count[q] > 0xFFFFFF)
+            return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: pool %d count %d", q, count[q]);
+        if (count[q] == 0) continue;
+        if (!base[q] || !aligned(base[q], 256))
+            return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: pool %d base must be non-NULL and "
+                        "256-byte aligned", q);
+        if (stride[q] < lay->bytes || stride[q] % 256)
+            return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: pool %d stride %lld (need >= %lld, "
+                        "multiple of 256)", q, (long long)stride[q], (long long)lay->bytes);
+    }
+    for (int e = 0; e < d->E; ++e) {
+        const uint32_t v = static_cast<uint32_t>(tb->pool_slot[e]);
+        const int q = (int)(v >> 31), slot = (int)(v & 0x7FFFFFFFu);
+        if (slot >= count[q])
+            return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: expert %d -> pool %d slot %d, but "
+                        "the pool has %d slots", e, q, slot, count[q]);
+    }
+    if (d->has_shared && (!tb->shared || !aligned(tb->shared, 256)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: shared expert image missing or "
+                    "not 256-byte aligned");
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace swb
+
+using namespace swb;
+
+extern "C" {
+
+size_t moe_grouped_ffn_workspace_size(const moe_ffn_desc* d) {
+    (void)d;
+    return 0;
+}
+
+moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, const void* x_perm,
+                           const float* x_perm_scales, const int32_t* offsets, void* h,
+                           void* y_perm, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    (void)x_perm_scales;
+    (void)workspace;
+    (void)workspace_bytes;
+    moe_expert_layout lay;
+    moe_status st = validate(d, tbl, &lay);
+    if (st != MOE_OK) return st;
+    if (d->T == 0) return MOE_OK;
+    if (!x_perm || !offsets || !h || !y_perm)
+        return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: NULL pointer");
+    if (!aligned(x_perm, 16) || !aligned(offsets, 16) || !aligned(h, 16) || !aligned(y_perm, 16))
+        return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: pointers must be 16-byte aligned");
+    const int64_t A = (int64_t)d->T * d->k;
+    const int64_t rows = A + (d->has_shared ? d->T : 0);
+    if (rows > INT32_MAX / 2) return fail(MOE_ERR_UNSUPPORTED, "moe_grouped_ffn: too many rows");
+    const int G = d->E + (d->has_shared ? 1 : 0);
+    int* err = nullptr;
+    st = device_error_word(&err);
+    if (st != MOE_OK) return st;
+
+    static thread_local FfnArgs a;  // ~5 KB: kept off the stack
+    memset(&a, 0, sizeof a);
+    a.offsets = offsets;
+    a.err = err;
+    a.E = d->E;
+    a.T = d->T;
+    a.A = (int32_t)A;
+    a.has_shared = d->has_shared ? 1 : 0;
+    for (int e = 0; e < d->E; ++e) a.pool_slot[e] = tbl->pool_slot[e];
+    const void* base[2] = {tbl->local_base, tbl->remote_base};
+    const int32_t count[2] = {tbl->local_count, tbl->remote_count};
+    const int64_t stride[2] = {tbl->local_stride, tbl->remote_stride};
+    const int bn = pick_bn(A, d->E);
+
+    // GEMM1: h = silu(X W_gate^T) * (X W_up^T)
+    for (int q = 0; q < 2; ++q)
+        if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.gu_offset, count[q],
+                                                    stride[q], d->H, 2 * d->I)) != MOE_OK)
+            return st;
+    if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.gu_offset, 1,
+                                                 lay.bytes, d->H, 2 * d->I)) != MOE_OK)
+        return st;
+    if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H)) != MOE_OK) return st;
+    a.K = d->H;
+    a.M = d->I;
+    a.up_row = d->I;
+    a.out = static_cast<__nv_bfloat16*>(h);
+    a.ld_out = d->I;
+    if ((st = launch_bn<true>(bn, a, (int)rows, G, stream)) != MOE_OK) return st;
+
+    // GEMM2: y = h W_down^T
+    for (int q = 0; q < 2; ++q)
+        if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.down_offset,
+                                                    count[q], stride[q], d->I, d->H)) != MOE_OK)
+            return st;
+    if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.down_offset, 1,
+                                                 lay.bytes, d->I, d->H)) != MOE_OK)
+        return st;
+    if ((st = encode_act_map(&a.act_map, h, rows, d->I)) != MOE_OK) return st;
+    a.K = d->I;
+    a.M = d->H;
+    a.up_row = 0;
+    a.out = static_cast<__nv_bfloat16*>(y_perm);
+    a.ld_out = d->H;
+    return launch_bn<false>(bn, a, (int)rows, G, stream);
+}
+
+}  // extern "C"

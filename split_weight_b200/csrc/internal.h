@@ -1,0 +1,55 @@
+// Host-side plumbing shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+
+#include "../../include/moe.h"
+
+namespace swb {
+
+// Records a thread-local message for moe_last_error() and returns `s`.
+moe_status fail(moe_status s, const char* fmt, ...);
+
+// Wraps every CUDA runtime call the library makes: honours the test hook
+// (moe_debug_fail_next_cuda_calls) and turns errors into MOE_ERR_CUDA.
+bool cuda_injected_failure();
+moe_status cuda_check(cudaError_t e, const char* what);
+
+#define SWB_CUDA(call)                                                          \
+    do {                                                                        \
+        if (::swb::cuda_injected_failure())                                     \
+            return ::swb::fail(MOE_ERR_CUDA, "%s: injected failure", #call);    \
+        cudaError_t _e = (call);                                                \
+        if (_e != cudaSuccess) return ::swb::cuda_check(_e, #call);             \
+    } while (0)
+
+// After a launch: report launch-configuration errors.
+#define SWB_LAUNCHED(what)                                                      \
+    do {                                                                        \
+        cudaError_t _e = cudaGetLastError();                                    \
+        if (_e != cudaSuccess) return ::swb::cuda_check(_e, what);              \
+    } while (0)
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Device address of the library's device error word on the current device.
+moe_status device_error_word(int** out);
+
+// Number of SMs of the current device (cached per device).
+moe_status sm_count(int* out);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda).
+moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, void* base,
+                        const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                        CUtensorMapSwizzle swizzle);
+
+// Bits of the device error word.
+enum : int { kDevErrTimeout = 1, kDevErrIndex = 2 };
+
+}  // namespace swb

@@ -1,0 +1,376 @@
+// moe_route: router logits (fp32 SIMT, fixed order), scores and top-k.
+//
+// The DWDP pages run DeepSeek-R1's MoE layer on every data-parallel rank
+// (arXiv 2604.01621, abstract) and state no router arithmetic; the routing
+// here is the DeepSeek-R1 layer shape read plainly (see include/moe.h).
+//
+// Logits are a dense [T,E] x [E,H]^T product, but they decide integers (the
+// selected experts), so they are computed on the CUDA cores in one defined
+// order that a CPU can reproduce bit for bit: chunks of 256 consecutive h,
+// each a chain of fused multiply-adds from 0, chunk sums added in ascending
+// order.  Tensor cores accumulate in an undefined order and are not used.
+#include <cuda_bf16.h>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace swb {
+namespace {
+
+constexpr int kChunk = 256;  // h per fused-multiply-add chain
+constexpr int kKT = 32;      // h per shared-memory tile
+
+__device__ __forceinline__ float load_x(const float* x, int64_t i) { return x[i]; }
+__device__ __forceinline__ float load_x(const __nv_bfloat16* x, int64_t i) {
+    return __bfloat162float(x[i]);
+}
+
+// Each thread owns a TM x TN block of (token, expert) pairs of a
+// (16 TM) x (16 TN) block tile.  With split != 0 the z index of the grid is
+// the chunk and the kernel writes that chunk's sum P_c to part[c][t][e];
+// otherwise it walks all chunks and writes l[t][e].
+template <typename XT, int TM, int TN>
+__global__ void __launch_bounds__(256) k_logits(const XT* __restrict__ x,
+                                                const float* __restrict__ wg, int T, int H, int E,
+                                                int split, float* __restrict__ out) {
+    constexpr int BT = 16 * TM, BE = 16 * TN;
+    __shared__ __align__(16) float xs[kKT][BT + 4];
+    __shared__ __align__(16) float ws[kKT][BE + 4];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int e0 = blockIdx.x * BE, t0 = blockIdx.y * BT;
+    int h_begin = 0, h_end = H;
+    if (split) {
+        h_begin = blockIdx.z * kChunk;
+        h_end = min(H, h_begin + kChunk);
+    }
+    float l[TM][TN], p[TM][TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) l[i][j] = p[i][j] = 0.0f;
+
+    for (int h0 = h_begin; h0 < h_end; h0 += kKT) {
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < BT * kKT; idx += 256) {
+            const int tt = idx / kKT, kk = idx % kKT, t = t0 + tt;
+            xs[kk][tt] = (t < T) ? load_x(x, (int64_t)t * H + h0 + kk) : 0.0f;
+        }
+        for (int idx = threadIdx.x; idx < BE * kKT; idx += 256) {
+            const int ee = idx / kKT, kk = idx % kKT, e = e0 + ee;
+            ws[kk][ee] = (e < E) ? wg[(int64_t)e * H + h0 + kk] : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kKT; ++kk) {
+            float a[TM], b[TN];
+#pragma unroll
+            for (int i = 0; i < TM; ++i) a[i] = xs[kk][ty * TM + i];
+#pragma unroll
+            for (int j = 0; j < TN; ++j) b[j] = ws[kk][tx * TN + j];
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < TN; ++j) p[i][j] = __fmaf_rn(a[i], b[j], p[i][j]);
+        }
+        const int h_next = h0 + kKT;
+        if (h_next % kChunk == 0 || h_next >= h_end) {  // a chunk ends here
+            const bool first = split || (h_next - 1) / kChunk == 0;
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < TN; ++j) {
+                    l[i][j] = first ? p[i][j] : __fadd_rn(l[i][j], p[i][j]);
+                    p[i][j] = 0.0f;
+                }
+        }
+    }
+    float* o = split ? out + (int64_t)blockIdx.z * T * E : out;
+#pragma unroll
+    for (int i = 0; i < TM; ++i) {
+        const int t = t0 + ty * TM + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < TN; ++j) {
+            const int e = e0 + tx * TN + j;
+            if (e < E) o[(int64_t)t * E + e] = l[i][j];
+        }
+    }
+}
+
+// e^y in fp64 for |y| <= 700, every step one IEEE operation: Cody-Waite
+// reduction with ln 2 = LN2_HI + LN2_LO (LN2_HI has 21 trailing zero bits),
+// Taylor polynomial to degree 13 by Horner, exact scaling by 2^n.
+// (W. J. Cody and W. Waite, Software Manual for the Elementary Functions.)
+__device__ __forceinline__ double exp64_cw(double y) {
+    const double kInvLn2 = 0x1.71547652b82fep+0;
+    const double kLn2Hi = 0x1.62e42fee00000p-1;
+    const double kLn2Lo = 0x1.a39ef35793c76p-33;
+    const double c[14] = {0x1.0000000000000p+0, 0x1.0000000000000p+0, 0x1.0000000000000p-1,
+                          0x1.5555555555555p-3, 0x1.5555555555555p-5, 0x1.1111111111111p-7,
+                          0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-16,
+                          0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
+                          0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};  // 1 / i!
+    const double n = rint(__dmul_rn(y, kInvLn2));
+    const double r = __dsub_rn(__dsub_rn(y, __dmul_rn(n, kLn2Hi)), __dmul_rn(n, kLn2Lo));
+    double p = c[13];
+#pragma unroll
+    for (int i = 12; i >= 0; --i) p = __dadd_rn(__dmul_rn(p, r), c[i]);
+    const long long e = static_cast<long long>(n) + 1023;
+    return __dmul_rn(p, __longlong_as_double(e << 52));
+}
+
+// fp32( 1 / (1 + e^-x) ) with x clamped to [-120, 40] (no fp32 result changes).
+__device__ __forceinline__ float sigmoid_f32(float l) {
+    const double x = fmin(fmax(static_cast<double>(l), -120.0), 40.0);
+    const double e = exp64_cw(-x);
+    return __double2float_rn(__ddiv_rn(1.0, __dadd_rn(1.0, e)));
+}
+
+__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+// Warp-wide best (key, index) pair; every lane gets the result.
+__device__ __forceinline__ void warp_best(float& k, int& i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float k2 = __shfl_xor_sync(0xffffffffu, k, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+        if (better(k2, i2, k, i)) {
+            k = k2;
+            i = i2;
+        }
+    }
+}
+
+// One warp per token.  Lane `lane` holds experts e = lane + 32 v.
+template <int V>
+__global__ void __launch_bounds__(256) k_select(const float* __restrict__ logits, int nsplit, int T,
+                                                int E, int k, int score, int n_group,
+                                                int topk_group, float routed_scale, int renorm,
+                                                const float* __restrict__ bias,
+                                                int32_t* __restrict__ topk_idx,
+                                                float* __restrict__ topk_w) {
+    __shared__ float keys_sh[8][32 * V];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    const float kNegInf = -__int_as_float(0x7f800000);
+    float lg[V], key[V], sc[V];
+    bool cand[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        const int e = lane + 32 * v;
+        lg[v] = kNegInf;
+        if (e < E) {
+            float acc = logits[(int64_t)t * E + e];
+            for (int c = 1; c < nsplit; ++c)
+                acc = __fadd_rn(acc, logits[((int64_t)c * T + t) * E + e]);
+            lg[v] = acc;
+        }
+        if (score == MOE_SCORE_SIGMOID) {
+            sc[v] = (e < E) ? sigmoid_f32(lg[v]) : 0.0f;
+            key[v] = (e < E) ? (bias ? __fadd_rn(sc[v], bias[e]) : sc[v]) : kNegInf;
+        } else {
+            sc[v] = lg[v];
+            key[v] = lg[v];
+        }
+        cand[v] = e < E;
+    }
+    // group-limited candidates
+    if (score == MOE_SCORE_SIGMOID && topk_group < n_group) {
+#pragma unroll
+        for (int v = 0; v < V; ++v) keys_sh[warp][lane + 32 * v] = key[v];
+        __syncwarp();
+        const int gs = E / n_group;
+        float gscore = kNegInf;
+        if (lane < n_group) {
+            float b1 = kNegInf, b2 = kNegInf;
+            for (int i = 0; i < gs; ++i) {
+                const float kv = keys_sh[warp][lane * gs + i];
+                if (kv > b1) {
+                    b2 = b1;
+                    b1 = kv;
+                } else if (kv > b2) {
+                    b2 = kv;
+                }
+            }
+            gscore = (gs == 1) ? b1 : __fadd_rn(b1, b2);
+        }
+        uint32_t gmask = 0;
+        float gk = gscore;
+        for (int s = 0; s < topk_group; ++s) {
+            float bk = (lane < n_group && !((gmask >> lane) & 1u)) ? gk : kNegInf;
+            int bi = (lane < n_group && !((gmask >> lane) & 1u)) ? lane : 0x7fffffff;
+            warp_best(bk, bi);
+            gmask |= 1u << bi;
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            const int e = lane + 32 * v;
+            cand[v] = cand[v] && ((gmask >> (e / gs)) & 1u);
+        }
+    }
+    // top-k, descending key, ties to the lower expert
+    int my_e = -1;
+    float my_s = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        float bk = kNegInf;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            const int e = lane + 32 * v;
+            if (cand[v] && better(key[v], e, bk, bi)) {
+                bk = key[v];
+                bi = e;
+            }
+        }
+        warp_best(bk, bi);
+        float s_sel = 0.0f;
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+            if (lane + 32 * v == bi) {
+                cand[v] = false;
+                s_sel = sc[v];
+            }
+        s_sel = __shfl_sync(0xffffffffu, s_sel, bi & 31);
+        if (lane == j) {
+            my_e = bi;
+            my_s = s_sel;
+        }
+    }
+    float w = 0.0f;
+    if (score == MOE_SCORE_SIGMOID) {
+        float d = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const float sj = __shfl_sync(0xffffffffu, my_s, j);
+            d = (j == 0) ? sj : __fadd_rn(d, sj);
+        }
+        w = renorm ? __fdiv_rn(my_s, d) : my_s;
+    } else {
+        const float lmax = __shfl_sync(0xffffffffu, my_s, 0);
+        const float num = (lane < k) ? expf(my_s - lmax) : 0.0f;
+        float den = 0.0f;
+        if (renorm) {
+            den = num;
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+                if (lane + 32 * v < E) den += expf(lg[v] - lmax);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        w = num / den;
+    }
+    if (lane < k) {
+        topk_idx[(int64_t)t * k + lane] = my_e;
+        topk_w[(int64_t)t * k + lane] = __fmul_rn(w, routed_scale);
+    }
+}
+
+struct RoutePlan {
+    int tm;      // 2 or 4 (TM == TN)
+    int nsplit;  // 1, or the number of 256-wide chunks
+};
+
+RoutePlan plan(const moe_route_cfg* c) {
+    RoutePlan p;
+    const int64_t tiles32 = (int64_t)((c->T + 31) / 32) * ((c->E + 31) / 32);
+    const bool small = tiles32 < 512;
+    p.tm = small ? 2 : 4;
+    p.nsplit = small ? (c->H + kChunk - 1) / kChunk : 1;
+    return p;
+}
+
+moe_status validate(const moe_route_cfg* c) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "moe_route: cfg is NULL");
+    if (c->T < 0 || c->H <= 0 || c->E <= 0 || c->k <= 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: T=%d H=%d E=%d k=%d", c->T, c->H, c->E, c->k);
+    if (c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK || c->k > c->E)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: E=%d (max %d), k=%d (max %d, <= E)", c->E,
+                    MOE_MAX_EXPERTS, c->k, MOE_MAX_TOPK);
+    if (c->H % 32) return fail(MOE_ERR_INVALID_ARG, "moe_route: H=%d not a multiple of 32", c->H);
+    if (c->score == MOE_SCORE_SIGMOID) {
+        if (c->n_group <= 0 || c->n_group > 32 || c->E % c->n_group)
+            return fail(MOE_ERR_INVALID_ARG, "moe_route: n_group=%d must divide E=%d, <= 32",
+                        c->n_group, c->E);
+        if (c->topk_group <= 0 || c->topk_group > c->n_group)
+            return fail(MOE_ERR_INVALID_ARG, "moe_route: topk_group=%d", c->topk_group);
+        if ((int64_t)c->k > (int64_t)c->topk_group * (c->E / c->n_group))
+            return fail(MOE_ERR_INVALID_ARG, "moe_route: k=%d exceeds the %d candidates", c->k,
+                        c->topk_group * (c->E / c->n_group));
+    } else if (c->score != MOE_SCORE_SOFTMAX) {
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: score=%d", c->score);
+    }
+    return MOE_OK;
+}
+
+template <typename XT>
+void launch_logits(const moe_route_cfg* c, const RoutePlan& p, const XT* x, const float* wg,
+                   float* out, cudaStream_t s) {
+    const int B = 16 * p.tm;
+    dim3 grid((c->E + B - 1) / B, (c->T + B - 1) / B, p.nsplit);
+    if (p.tm == 2)
+        k_logits<XT, 2, 2><<<grid, 256, 0, s>>>(x, wg, c->T, c->H, c->E, p.nsplit > 1, out);
+    else
+        k_logits<XT, 4, 4><<<grid, 256, 0, s>>>(x, wg, c->T, c->H, c->E, p.nsplit > 1, out);
+}
+
+}  // namespace
+}  // namespace swb
+
+using namespace swb;
+
+extern "C" {
+
+size_t moe_route_workspace_size(const moe_route_cfg* c) {
+    if (validate(c) != MOE_OK) return 0;
+    const RoutePlan p = plan(c);
+    return (size_t)p.nsplit * c->T * c->E * sizeof(float);
+}
+
+moe_status moe_route(const moe_route_cfg* c, const void* x, moe_dtype x_dtype, const float* w_gate,
+                     const float* bias, int32_t* topk_idx, float* topk_w, void* workspace,
+                     size_t workspace_bytes, cudaStream_t stream) {
+    moe_status st = validate(c);
+    if (st != MOE_OK) return st;
+    if (x_dtype != MOE_F32 && x_dtype != MOE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "moe_route: x dtype %d", (int)x_dtype);
+    if (c->T == 0) return MOE_OK;
+    if (!x || !w_gate || !topk_idx || !topk_w)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: NULL pointer");
+    if (bias && c->score != MOE_SCORE_SIGMOID)
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: bias is only defined for sigmoid scores");
+    if (!aligned(x, 16) || !aligned(w_gate, 16) || !aligned(topk_idx, 16) ||
+        !aligned(topk_w, 16) || (bias && !aligned(bias, 16)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: pointers must be 16-byte aligned");
+    const size_t need = moe_route_workspace_size(c);
+    if (workspace_bytes < need || (need && !workspace))
+        return fail(MOE_ERR_WORKSPACE, "moe_route: workspace %zu < %zu bytes", workspace_bytes,
+                    need);
+    if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "moe_route: injected failure");
+    const RoutePlan p = plan(c);
+    float* lg = static_cast<float*>(workspace);
+    if (x_dtype == MOE_F32)
+        launch_logits(c, p, static_cast<const float*>(x), w_gate, lg, stream);
+    else
+        launch_logits(c, p, static_cast<const __nv_bfloat16*>(x), w_gate, lg, stream);
+    SWB_LAUNCHED("moe_route: logits kernel");
+    const int blocks = (c->T + 7) / 8;
+    const int V = (c->E + 31) / 32;
+#define SWB_SELECT(VV)                                                                        \
+    k_select<VV><<<blocks, 256, 0, stream>>>(lg, p.nsplit, c->T, c->E, c->k, c->score,        \
+                                             c->n_group, c->topk_group, c->routed_scale,      \
+                                             c->renormalize, bias, topk_idx, topk_w)
+    if (V <= 1) SWB_SELECT(1);
+    else if (V <= 2) SWB_SELECT(2);
+    else if (V <= 4) SWB_SELECT(4);
+    else if (V <= 8) SWB_SELECT(8);
+    else if (V <= 16) SWB_SELECT(16);
+    else SWB_SELECT(32);
+#undef SWB_SELECT
+    SWB_LAUNCHED("moe_route: select kernel");
+    return MOE_OK;
+}
+
+}  // extern "C"

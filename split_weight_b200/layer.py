@@ -1,0 +1,247 @@
+"""Layer-level driver of the C ABI: one DWDP rank's MoE block.
+
+``MoELayer.forward`` enqueues moe_route -> moe_permute -> moe_grouped_ffn ->
+moe_combine on one stream.  torch provides device memory, streams and events
+only; every step of the block runs in libswb_moe.so.
+
+``SplitWeights`` holds one layer's expert weights in two pools that have
+nothing to do with each other in memory - the rank's own experts (local)
+and the buffer the remote experts were fetched into - plus the per-expert
+(pool, slot) table through which the grouped GEMM finds each expert (the
+split-weight figure of the explainer "Distributed Weight Data Parallelism
+cuts LLM inference stalls": no merge into one contiguous buffer).
+``PrefetchPipeline`` runs several layers with the next layers' remote
+experts copied into alternate buffers on a copy-engine stream (the
+explainer's prefetch figure).
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import _lib as L
+
+POOL_LOCAL, POOL_REMOTE = 0, 1
+_DT = {"f32": L.MOE_F32, "bf16": L.MOE_BF16, "e4m3": L.MOE_E4M3}
+
+
+@dataclass(frozen=True)
+class LayerShape:
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    score: str = "sigmoid"       # "softmax" | "sigmoid"
+    n_group: int = 1
+    topk_group: int = 1
+    routed_scale: float = 1.0
+    renormalize: bool = True
+    has_shared: bool = False
+    x_dtype: str = "bf16"        # "f32" | "bf16"
+    w_dtype: str = "bf16"        # "bf16" | "e4m3"
+    y_dtype: str = "bf16"        # "f32" | "bf16"
+
+    @property
+    def A(self) -> int:
+        return self.T * self.k
+
+    @property
+    def rows(self) -> int:
+        return self.A + (self.T if self.has_shared else 0)
+
+    def route_cfg(self) -> L.moe_route_cfg:
+        return L.moe_route_cfg(self.T, self.H, self.E, self.k,
+                               L.MOE_SCORE_SIGMOID if self.score == "sigmoid" else L.MOE_SCORE_SOFTMAX,
+                               self.n_group, self.topk_group, self.routed_scale,
+                               1 if self.renormalize else 0)
+
+    def ffn_desc(self) -> L.moe_ffn_desc:
+        return L.moe_ffn_desc(self.T, self.H, self.I, self.E, self.k, _DT[self.w_dtype],
+                              L.MOE_BF16, 1 if self.has_shared else 0)
+
+
+def _stream_handle(stream: torch.cuda.Stream | None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+class SplitWeights:
+    """Expert weights of one layer split over a local and a remote pool."""
+
+    def __init__(self, H: int, I: int, w_dtype: str, pool_slot: np.ndarray, local: torch.Tensor,
+                 n_local: int, remote: torch.Tensor, n_remote: int, shared: torch.Tensor | None):
+        self.H, self.I, self.w_dtype = H, I, w_dtype
+        self.layout = L.expert_layout(H, I, _DT[w_dtype])
+        self.stride = int(self.layout.bytes)
+        self.pool_slot = np.ascontiguousarray(pool_slot, dtype=np.int32)
+        self.local, self.n_local = local, n_local
+        self.remote, self.n_remote = remote, n_remote
+        self.shared = shared
+
+    @staticmethod
+    def image_bytes(H: int, I: int, w_dtype: str) -> int:
+        return int(L.expert_layout(H, I, _DT[w_dtype]).bytes)
+
+    @classmethod
+    def allocate(cls, H, I, w_dtype, pool_of, slot_of, has_shared, device) -> "SplitWeights":
+        """Empty pools sized for the given assignment of experts to (pool, slot)."""
+        pool_of = np.asarray(pool_of)
+        slot_of = np.asarray(slot_of)
+        n_local = int((pool_of == POOL_LOCAL).sum())
+        n_remote = int((pool_of == POOL_REMOTE).sum())
+        b = cls.image_bytes(H, I, w_dtype)
+        local = torch.empty(max(n_local, 1) * b, dtype=torch.uint8, device=device)
+        remote = torch.empty(max(n_remote, 1) * b, dtype=torch.uint8, device=device)
+        shared = torch.empty(b, dtype=torch.uint8, device=device) if has_shared else None
+        ps = (pool_of.astype(np.int64) << 31 | slot_of.astype(np.int64)).astype(np.uint32).view(np.int32)
+        return cls(H, I, w_dtype, ps, local, n_local, remote, n_remote, shared)
+
+    def slot_base(self, pool: int, slot: int) -> int:
+        t = self.local if pool == POOL_LOCAL else self.remote
+        return t.data_ptr() + slot * self.stride
+
+    def expert_base(self, e: int) -> int:
+        """Device address of expert e's image (e == E: the shared expert)."""
+        if e == len(self.pool_slot):
+            return self.shared.data_ptr()
+        v = int(np.uint32(self.pool_slot[e]))
+        return self.slot_base(v >> 31, v & 0x7FFFFFFF)
+
+    def table(self, remote: torch.Tensor | None = None) -> L.moe_expert_table:
+        """C table; `remote` overrides the remote pool (an alternate buffer)."""
+        rem = self.remote if remote is None else remote
+        self._ps_c = self.pool_slot.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        return L.moe_expert_table(self.local.data_ptr(), self.n_local, self.stride,
+                                  rem.data_ptr(), self.n_remote, self.stride,
+                                  _ptr(self.shared), self._ps_c)
+
+
+class MoELayer:
+    """One MoE layer with preallocated device buffers."""
+
+    def __init__(self, shape: LayerShape, w_gate: torch.Tensor, bias: torch.Tensor | None,
+                 weights: SplitWeights, device: torch.device | str = "cuda"):
+        s = shape
+        self.shape, self.w_gate, self.bias, self.weights = s, w_gate, bias, weights
+        dev = torch.device(device)
+        self._cfg = s.route_cfg()
+        self._desc = s.ffn_desc()
+        i32 = torch.int32
+        self.route_ws = torch.empty(max(L.moe_route_workspace_size(ctypes.byref(self._cfg)), 16),
+                                    dtype=torch.uint8, device=dev)
+        self.perm_ws = torch.empty(max(L.moe_permute_workspace_size(s.T, s.k, s.E), 16),
+                                   dtype=torch.uint8, device=dev)
+        self.topk_idx = torch.empty(max(s.T, 1), s.k, dtype=i32, device=dev)
+        self.topk_w = torch.empty(max(s.T, 1), s.k, dtype=torch.float32, device=dev)
+        self.offsets = torch.empty(s.E + 1, dtype=i32, device=dev)
+        self.perm_src = torch.empty(max(s.A, 1), dtype=i32, device=dev)
+        self.inv_pos = torch.empty(max(s.T, 1), s.k, dtype=i32, device=dev)
+        rows = max(s.rows, 1)
+        self.x_perm = torch.empty(rows, s.H, dtype=torch.bfloat16, device=dev)
+        self.h = torch.empty(rows, s.I, dtype=torch.bfloat16, device=dev)
+        self.y_perm = torch.empty(rows, s.H, dtype=torch.bfloat16, device=dev)
+        ydt = torch.float32 if s.y_dtype == "f32" else torch.bfloat16
+        self.y = torch.empty(max(s.T, 1), s.H, dtype=ydt, device=dev)
+
+    # -- the four steps, each one C-ABI call ---------------------------------
+    def route(self, x: torch.Tensor, stream: int) -> None:
+        L.check(L.moe_route(ctypes.byref(self._cfg), x.data_ptr(), _DT[self.shape.x_dtype],
+                            self.w_gate.data_ptr(), _ptr(self.bias), self.topk_idx.data_ptr(),
+                            self.topk_w.data_ptr(), self.route_ws.data_ptr(),
+                            self.route_ws.numel(), stream))
+
+    def permute(self, x: torch.Tensor, stream: int) -> None:
+        s = self.shape
+        L.check(L.moe_permute(s.T, s.k, s.E, s.H, self.topk_idx.data_ptr(), x.data_ptr(),
+                              _DT[s.x_dtype], L.MOE_BF16, 1 if s.has_shared else 0,
+                              self.offsets.data_ptr(), self.perm_src.data_ptr(),
+                              self.inv_pos.data_ptr(), self.x_perm.data_ptr(), None,
+                              self.perm_ws.data_ptr(), self.perm_ws.numel(), stream))
+
+    def grouped_ffn(self, stream: int, remote: torch.Tensor | None = None) -> None:
+        tbl = self.weights.table(remote)
+        L.check(L.moe_grouped_ffn(ctypes.byref(self._desc), ctypes.byref(tbl),
+                                  self.x_perm.data_ptr(), None, self.offsets.data_ptr(),
+                                  self.h.data_ptr(), self.y_perm.data_ptr(), None, 0, stream))
+
+    def combine(self, stream: int) -> None:
+        s = self.shape
+        L.check(L.moe_combine(s.T, s.k, s.H, self.y_perm.data_ptr(), self.inv_pos.data_ptr(),
+                              self.topk_w.data_ptr(), 1 if s.has_shared else 0, self.y.data_ptr(),
+                              _DT[s.y_dtype], stream))
+
+    def forward(self, x: torch.Tensor, stream: torch.cuda.Stream | None = None,
+                remote: torch.Tensor | None = None) -> torch.Tensor:
+        """Enqueues the whole block on `stream`; returns the output buffer."""
+        h = _stream_handle(stream)
+        self.route(x, h)
+        self.permute(x, h)
+        self.grouped_ffn(h, remote)
+        self.combine(h)
+        return self.y
+
+
+class PrefetchPipeline:
+    """Consecutive MoE layers whose remote experts are fetched ahead into two
+    alternate buffers by moe_prefetch_layer on a copy-engine stream.
+
+    Layer l computes from remote_bufs[l % 2]; as soon as layer l's grouped
+    GEMMs have been enqueued, the copy stream waits for them (free event) and
+    starts fetching layer l + 2 into the same buffer.  Layer l waits for its
+    own ready event before its grouped GEMM.
+    """
+
+    def __init__(self, layers: list[MoELayer], peer_stores: list[torch.Tensor],
+                 remote_bytes: int, device: torch.device | str = "cuda", chunk_bytes: int = 0):
+        self.layers, self.peer_stores = layers, peer_stores
+        self.remote_bytes, self.chunk_bytes = remote_bytes, chunk_bytes
+        dev = torch.device(device)
+        self.bufs = [torch.empty(max(remote_bytes, 1), dtype=torch.uint8, device=dev)
+                     for _ in range(min(2, len(layers)))]
+        self.copy_stream = torch.cuda.Stream(device=dev)
+        self.ready = [torch.cuda.Event() for _ in layers]
+        self.free = [torch.cuda.Event() for _ in self.bufs]
+
+    def _prefetch(self, l: int, wait_free: torch.cuda.Event | None) -> None:
+        L.check(L.moe_prefetch_layer(self.peer_stores[l].data_ptr(), self.bufs[l % 2].data_ptr(),
+                                     self.remote_bytes, self.chunk_bytes,
+                                     self.copy_stream.cuda_stream,
+                                     wait_free.cuda_event if wait_free is not None else None,
+                                     self.ready[l].cuda_event))
+
+    def prime(self) -> None:
+        """Enqueues the fetch of the first two layers (before the timed loop)."""
+        for l in range(len(self.bufs)):
+            self._prefetch(l, None)
+
+    def run(self, xs: list[torch.Tensor], stream: torch.cuda.Stream | None = None,
+            prefetch: bool = True, wrap: bool = True) -> list[torch.Tensor]:
+        """Runs all layers.  With prefetch=False the buffers are used as they
+        are (nothing is copied).  With wrap=True the fetches issued during the
+        last layers are those of the next pass's first layers, as in a
+        steady stream of forward passes; prime() must have run once."""
+        stream = stream if stream is not None else torch.cuda.current_stream()
+        h = stream.cuda_stream
+        outs = []
+        n = len(self.layers)
+        for l, layer in enumerate(self.layers):
+            layer.route(xs[l], h)
+            layer.permute(xs[l], h)
+            if prefetch:
+                stream.wait_event(self.ready[l])
+            layer.grouped_ffn(h, self.bufs[l % 2])
+            nxt = l + 2
+            if prefetch and (nxt < n or (wrap and n >= 2)):
+                self.free[l % 2].record(stream)
+                self._prefetch(nxt % n, self.free[l % 2])
+            layer.combine(h)
+            outs.append(layer.y)
+        return outs

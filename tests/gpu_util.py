@@ -1,0 +1,52 @@
+"""Helpers shared by the GPU tests (device workloads + oracle references)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from moe_inputs import config, device as mdev
+
+# Floating-point bar: max |gpu - oracle| <= RTOL_BF16 * max |oracle| over the
+# compared outputs (bf16 weights and activations, fp32 accumulation; the GPU
+# rounds x_perm, h and y_perm to bf16 while the oracle keeps fp64).
+RTOL_BF16 = 2e-2
+RTOL_FP8 = 6e-2
+
+# Test-only workloads: same recipes, other sizes (own generator keys).
+MID_SIGMOID = config(2).with_(cfg_id=11, name="mid_sigmoid_T300_H512_I256_E32", T=300, H=512,
+                              I=256, E=32, k=4, n_group=4, topk_group=2, local_count=8)
+MID_SOFTMAX = config(1).with_(cfg_id=12, name="mid_softmax_f32_T257_H384_I256_E16", T=257, H=384,
+                              I=256, E=16, k=3, local_count=6)
+SPARSE_DECODE = config(2).with_(cfg_id=13, name="sparse_decode_T5_H256_I128_E64", T=5, H=256,
+                                I=128, E=64, k=8, n_group=8, topk_group=4, local_count=16)
+ONE_TOKEN = config(2).with_(cfg_id=14, name="one_token_H256_I256_E16", T=1, H=256, I=256, E=16,
+                            k=2, n_group=4, topk_group=2, local_count=4)
+
+
+def sync_check():
+    from split_weight_b200 import _lib as L
+    torch.cuda.synchronize()
+    L.check(L.moe_check_device())
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return t.float().cpu().numpy().astype(np.float64)
+    return t.cpu().numpy()
+
+
+def assert_close_rel(got: np.ndarray, ref: np.ndarray, rtol: float, what: str):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    scale = np.abs(ref).max()
+    err = np.abs(got - ref).max()
+    assert err <= rtol * scale, f"{what}: max|err| {err:.4g} > {rtol} * max|ref| {scale:.4g}"
+    return err / scale
+
+
+def run_layer(dl: mdev.DeviceLayer):
+    dl.layer.forward(dl.x)
+    sync_check()
+    return dl.layer

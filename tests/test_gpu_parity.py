@@ -1,0 +1,167 @@
+"""GPU parity: every C-ABI call against the CPU oracle on the same seeded inputs.
+
+Routing indices, counts, offsets and the permutation must be bit-exact; the
+sigmoid routing weights too (their arithmetic is defined in fp32).  Layer
+outputs must satisfy max|err| <= 2e-2 * max|ref| (bf16 path).
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_inputs import config, device as mdev, gen
+from oracle import workload as ow
+from split_weight_b200 import _lib as L
+
+from gpu_util import (MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16, SPARSE_DECODE,
+                      assert_close_rel, run_layer, sync_check, to_np)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [config(1), MID_SIGMOID, MID_SOFTMAX, SPARSE_DECODE, ONE_TOKEN]
+
+
+@pytest.fixture(autouse=True)
+def _free_memory(cuda_device):
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def _check_routing(dl, idx_ref, w_ref):
+    ml = dl.layer
+    T = dl.cfg.T
+    idx = ml.topk_idx[:T].cpu().numpy()
+    np.testing.assert_array_equal(idx, idx_ref, err_msg="topk_idx differs from the oracle")
+    w = ml.topk_w[:T].cpu().numpy()
+    if dl.cfg.score == "sigmoid":
+        np.testing.assert_array_equal(w, w_ref.astype(np.float32), err_msg="topk_w not bit-exact")
+    else:
+        np.testing.assert_allclose(w, w_ref, rtol=2e-6, atol=1e-7)
+
+
+def _check_permutation(dl, idx_ref):
+    ml, c = dl.layer, dl.cfg
+    off, src, inv = oracle.permute(idx_ref, c.E)
+    np.testing.assert_array_equal(ml.offsets.cpu().numpy(), off)
+    np.testing.assert_array_equal(ml.perm_src[:c.A].cpu().numpy(), src)
+    np.testing.assert_array_equal(ml.inv_pos[:c.T].cpu().numpy(), inv)
+    # gathered rows: x (rounded to bf16 when it came as fp32), then the shared rows
+    xp = ml.x_perm[:c.rows].view(torch.int16).cpu().numpy().view(np.uint16)
+    xb = gen.f32_to_bf16_bits(dl.inputs.x)
+    np.testing.assert_array_equal(xp[:c.A], xb[src])
+    if c.has_shared:
+        np.testing.assert_array_equal(xp[c.A:], xb)
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_small_layer_full_parity(cfg):
+    dl = mdev.build_layer(cfg)
+    run_layer(dl)
+    y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
+    _check_routing(dl, idx_ref, w_ref)
+    _check_permutation(dl, idx_ref)
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, RTOL_BF16, f"{cfg.name} y")
+
+
+def test_generator_gpu_matches_host(cuda_device):
+    for cfg in (config(2), config(5).with_(H=512, I=256)):
+        lay = L.expert_layout(cfg.H, cfg.I, L.MOE_E4M3 if cfg.w_dtype == "e4m3" else L.MOE_BF16)
+        buf = torch.empty(lay.bytes, dtype=torch.uint8, device=cuda_device)
+        from moe_inputs import gpu_gen
+        base = buf.data_ptr()
+        gsc = base + lay.gu_scale_offset if lay.gu_scale_offset >= 0 else None
+        dsc = base + lay.down_scale_offset if lay.down_scale_offset >= 0 else None
+        gpu_gen.fill_expert(cfg, 0, 7, base + lay.gu_offset, base + lay.down_offset, gsc, dsc,
+                            torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        host = gen.expert_host(cfg, 0, 7)
+        raw = buf.cpu().numpy()
+        esz = 2 if cfg.w_dtype == "bf16" else 1
+        gu = raw[lay.gu_offset: lay.gu_offset + host.gu.size * esz].view(host.gu.dtype)
+        np.testing.assert_array_equal(gu.reshape(host.gu.shape), host.gu)
+        dn = raw[lay.down_offset: lay.down_offset + host.down.size * esz].view(host.down.dtype)
+        np.testing.assert_array_equal(dn.reshape(host.down.shape), host.down)
+        if host.gu_scale is not None:
+            s = raw[lay.gu_scale_offset: lay.gu_scale_offset + host.gu_scale.size * 4].view(np.float32)
+            np.testing.assert_array_equal(s.reshape(host.gu_scale.shape), host.gu_scale)
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_pool_invariance_bit_identical(seed):
+    cfg = MID_SIGMOID
+    ref_dl = mdev.build_layer(cfg)
+    y_ref = run_layer(ref_dl).y.clone()
+    del ref_dl
+    for n_local in (None, 0, cfg.E):
+        pl = mdev.random_placement(cfg, seed, n_local)
+        dl = mdev.build_layer(cfg, placement=pl)
+        y = run_layer(dl).y
+        assert torch.equal(y, y_ref), f"placement {pl} changed the output"
+
+
+def test_all_tokens_one_expert_is_dense_ffn():
+    # a large bias on one expert and k = 1: every token goes to expert 5, the
+    # grouped GEMM sees one dense group spanning several token tiles
+    cfg = MID_SIGMOID.with_(cfg_id=15, k=1, topk_group=1, has_shared=False)
+    dl = mdev.build_layer(cfg)
+    b = dl.layer.bias.clone()
+    b[5] = 10.0
+    dl.layer.bias.copy_(b)
+    dl.inputs.bias = b.cpu().numpy()
+    run_layer(dl)
+    assert (dl.layer.topk_idx[:cfg.T] == 5).all()
+    y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
+    assert (idx_ref == 5).all()
+    _check_routing(dl, idx_ref, w_ref)
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, RTOL_BF16, "dense y")
+
+
+def test_empty_batch_is_a_no_op(cuda_device):
+    cfg = MID_SIGMOID.with_(cfg_id=16, T=0)
+    dl = mdev.build_layer(cfg)
+    dl.layer.forward(dl.x)
+    sync_check()
+    assert dl.layer.offsets.cpu().numpy().tolist() == [0] * (cfg.E + 1)
+
+
+def test_out_of_range_expert_index_is_reported(cuda_device):
+    cfg = SPARSE_DECODE
+    dl = mdev.build_layer(cfg)
+    ml = dl.layer
+    h = torch.cuda.current_stream().cuda_stream
+    ml.route(dl.x, h)
+    ml.topk_idx[0, 0] = cfg.E + 3   # made on the host side: the kernel checks and skips it
+    ml.permute(dl.x, h)
+    torch.cuda.synchronize()
+    assert L.moe_check_device() == L.MOE_ERR_DEVICE_CHECK
+    assert L.moe_check_device() == L.MOE_OK   # the word was cleared
+
+
+# ----------------------------------------------------------------- full size
+def _full_size_check(cfg, layer: int, n_sample: int = 12):
+    dl = mdev.build_layer(cfg, layer=layer)
+    run_layer(dl)
+    idx_ref, w_ref, _ = ow.route(cfg, layer, dl.inputs)
+    _check_routing(dl, idx_ref, w_ref)
+    _check_permutation(dl, idx_ref)
+    rng = np.random.default_rng(100 + layer)
+    toks = np.sort(rng.choice(cfg.T, size=min(n_sample, cfg.T), replace=False))
+    y_ref = ow.layer_tokens(cfg, layer, toks, idx_ref, w_ref, dl.pool, dl.slot, dl.inputs)
+    y = to_np(dl.layer.y[torch.from_numpy(toks).cuda()])
+    return assert_close_rel(y, y_ref, RTOL_BF16, f"{cfg.name} layer {layer} sampled y")
+
+
+def test_r1_decode_full_size():
+    _full_size_check(config(2), 0, n_sample=16)
+
+
+def test_r1_prefill_8k_full_size():
+    _full_size_check(config(3), 0, n_sample=8)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_r1_prefill_imbalanced_full_size(layer):
+    _full_size_check(config(4), layer, n_sample=6)
