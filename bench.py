@@ -1,0 +1,515 @@
+#!/usr/bin/env python3
+"""MoE-layer throughput of one DWDP rank's MoE block (tokens/s) and the
+roofline fraction of its grouped expert GEMM.
+
+A step is one pass of the whole block over one batch: router + top-k,
+permutation, grouped SwiGLU FFN over the split (local + remote) expert
+pools, combine - and, for the multi-layer pipelined workloads, the
+copy-engine prefetch of later layers' remote experts into the alternate
+buffers.  Default workload: the DeepSeek-R1-shaped decode step (128 tokens,
+H=7168, I=2048, 256 routed experts + 1 shared, top-8 of 8 groups / top-4,
+bf16 weights, 64 local / 192 remote experts).
+
+  python bench.py [--gpus N --steps K --warmup W] [--config 1..5] [--impl reference]
+
+N > 1 (torchrun): N independent data-parallel replicas, one per GPU (the
+block has no collective; each rank runs its own tokens): weak scaling,
+value = tokens of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at DeepSeek-R1 shape; % of HBM/tensor roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_LAYER = 9  # route 2 + permute 4 + grouped FFN 2 + combine 1
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "grouped_ffn_traffic.json")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--config", type=int, default=2)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args(argv)
+
+
+# ----------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("ffn.cu", "device.cuh"):
+        with open(os.path.join(ROOT, "split_weight_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the grouped FFN from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_call")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while it runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def workload_desc(cfg) -> str:
+    d = (f"{cfg.name}: T={cfg.T} tokens x {cfg.layers} layer(s), H={cfg.H}, I={cfg.I}, "
+         f"E={cfg.E} routed" + (" + 1 shared" if cfg.has_shared else "") + f", top-{cfg.k} {cfg.score}")
+    if cfg.score == "sigmoid":
+        d += f" ({cfg.n_group} groups / top-{cfg.topk_group})"
+    d += f", {cfg.w_dtype} weights, {cfg.local_count} local / {cfg.E - cfg.local_count} remote experts"
+    return d
+
+
+def roofline_figures(cfg, counts_per_layer, peaks):
+    """Algorithmic FLOPs and bytes of the grouped FFN per step."""
+    wbytes = 2 if cfg.w_dtype == "bf16" else 1
+    act = 2
+    flops = 0.0
+    nbytes = 0.0
+    for counts in counts_per_layer:
+        touched = int((np.asarray(counts) > 0).sum()) + (1 if cfg.has_shared else 0)
+        rows = cfg.A + (cfg.T if cfg.has_shared else 0)
+        flops += rows * 6.0 * cfg.H * cfg.I
+        nbytes += touched * 3.0 * cfg.H * cfg.I * wbytes + 2.0 * cfg.T * cfg.H * act
+    return flops, nbytes
+
+
+# ----------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from moe_inputs import config, device as mdev
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = config(args.config)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+
+    # ---- workload (resident in HBM before timing)
+    dls = [mdev.build_layer(cfg, layer=l, device=dev) for l in range(cfg.layers)]
+    pipe = None
+    if cfg.layers > 1:
+        from split_weight_b200 import PrefetchPipeline
+        stores = [mdev.peer_store(cfg, l, dls[l].layer.weights, dev) for l in range(cfg.layers)]
+        rbytes = dls[0].layer.weights.n_remote * dls[0].layer.weights.stride
+        pipe = PrefetchPipeline([d.layer for d in dls], stores, rbytes, dev)
+        for d in dls:  # the layers' own remote pools are not needed: the buffers replace them
+            d.layer.weights.remote = torch.empty(1, dtype=torch.uint8, device=dev)
+        torch.cuda.empty_cache()
+        pipe.prime()
+    torch.cuda.synchronize()
+
+    xs = [d.x for d in dls]
+    h = stream.cuda_stream
+
+    def step(timed_ffn=None, prefetch=True):
+        if pipe is None:
+            ml = dls[0].layer
+            ml.route(xs[0], h)
+            ml.permute(xs[0], h)
+            if timed_ffn is not None:
+                timed_ffn[0][0].record(stream)
+            ml.grouped_ffn(h)
+            if timed_ffn is not None:
+                timed_ffn[0][1].record(stream)
+            ml.combine(h)
+            return
+        n = cfg.layers
+        for l, d in enumerate(dls):
+            ml = d.layer
+            ml.route(xs[l], h)
+            ml.permute(xs[l], h)
+            if prefetch:
+                stream.wait_event(pipe.ready[l])
+            if timed_ffn is not None:
+                timed_ffn[l][0].record(stream)
+            ml.grouped_ffn(h, pipe.bufs[l % 2])
+            if timed_ffn is not None:
+                timed_ffn[l][1].record(stream)
+            if prefetch:
+                pipe.free[l % 2].record(stream)
+                pipe._prefetch((l + 2) % n, pipe.free[l % 2])
+            ml.combine(h)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    from split_weight_b200 import _lib as L
+    L.check(L.moe_check_device())
+    counts = [np.diff(d.layer.offsets.cpu().numpy()) for d in dls]
+
+    # ---- device-timed region (FFN launches bracketed by their own events)
+    def events(n):
+        return [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(cfg.layers)] for _ in range(n)]
+    ffn_ev = events(args.steps)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(ffn_ev[i])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    ffn_ms = sum(a.elapsed_time(b) for st in ffn_ev for a, b in st) / args.steps
+    barrier()
+    L.check(L.moe_check_device())
+
+    # ---- pipelined workloads: exposed copy time per layer
+    prefetch_info = None
+    if pipe is not None:
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(reps):
+            step(prefetch=False)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        nocopy_ms = e0.elapsed_time(e1) / reps
+        # copy alone
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(pipe.copy_stream)
+        pipe._prefetch(0, None)
+        c1.record(pipe.copy_stream)
+        torch.cuda.synchronize()
+        copy_ms = c0.elapsed_time(c1)
+        pipe.prime()
+        torch.cuda.synchronize()
+        piped_ms = elapsed_ms / args.steps
+        exposed = max(0.0, (piped_ms - nocopy_ms) / cfg.layers)
+        prefetch_info = {
+            "remote_bytes_per_layer": pipe.remote_bytes,
+            "copy_alone_ms_per_layer": round(copy_ms, 4),
+            "step_ms_pipelined": round(piped_ms, 4),
+            "step_ms_no_copy": round(nocopy_ms, 4),
+            "exposed_copy_ms_per_layer": round(exposed, 4),
+            "hidden_fraction": round(1.0 - exposed / copy_ms, 4) if copy_ms > 0 else None,
+        }
+
+    # ---- end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_host = [d.x.cpu().pin_memory() for d in dls]
+        y_host = [torch.empty_like(d.layer.y[:cfg.T], device="cpu").pin_memory() for d in dls]
+        for _ in range(2):
+            for l, d in enumerate(dls):
+                xs[l].copy_(x_host[l], non_blocking=True)
+            step()
+            for l, d in enumerate(dls):
+                y_host[l].copy_(d.layer.y[:cfg.T], non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record(stream)
+        for _ in range(args.steps):
+            for l in range(cfg.layers):
+                xs[l].copy_(x_host[l], non_blocking=True)
+            step()
+            for l, d in enumerate(dls):
+                y_host[l].copy_(d.layer.y[:cfg.T], non_blocking=True)
+        q1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(q0.elapsed_time(q1), world, dev)
+        h2d = sum(t.numel() * t.element_size() for t in x_host)
+        d2h = sum(t.numel() * t.element_size() for t in y_host)
+        e2e = {"value": None, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "_ms": e2e_ms}
+    barrier()
+
+    max_ms = max_over_ranks(elapsed_ms, world, dev)
+    tokens_per_step = cfg.T * cfg.layers
+    total_tokens = sum_over_ranks(tokens_per_step * args.steps, world, dev)
+    value = total_tokens / (max_ms / 1e3)
+    if e2e is not None:
+        e2e["value"] = round(total_tokens / (e2e.pop("_ms") / 1e3), 3)
+
+    peaks, peak_src = load_peaks()
+    flops, nbytes = roofline_figures(cfg, counts, peaks)
+    hbm = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    if cfg.w_dtype == "e4m3":
+        tc_peak *= 2.0  # fp8 dense = 2x bf16 (nominal ratio)
+    t_hbm = nbytes / (hbm * 1e9)
+    t_flop = flops / (tc_peak * 1e12)
+    ffn_s = ffn_ms / 1e3
+    workload = cfg.name
+    if t_hbm >= t_flop:
+        achieved = nbytes / ffn_s / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4)}
+    else:
+        achieved = flops / ffn_s / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4)}
+    traffic = profiled_traffic(workload)
+    roof.update({
+        "traffic": (traffic * cfg.layers if traffic is not None else None),
+        "kernel": "moe_grouped_ffn (gate/up + down launches)",
+        "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
+        "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+        "kernel_ms_per_step": round(ffn_ms, 4),
+        "roof_ms_per_step": round(max(t_hbm, t_flop) * 1e3, 4),
+        "frac_of_roof": round(max(t_hbm, t_flop) / ffn_s, 4),
+    })
+
+    clocks = clk.summary() if rank == 0 else None
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.w_dtype, "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "tokens_per_rank_per_step": tokens_per_step,
+                   "layers": cfg.layers, "parallelism": f"dp{world} replicas (no collective)",
+                   "l2": "inputs larger than L2: %.1f GB of expert weights per step" % (nbytes / 1e9)},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": LAUNCHES_PER_LAYER * cfg.layers * args.steps,
+        "clocks": clocks,
+    }
+    if prefetch_info is not None:
+        out["prefetch"] = prefetch_info
+    return out, cfg
+
+
+# ----------------------------------------------------------------------- oracle
+def oracle_sample(cfg, n_tokens: int, reps: int = 1):
+    """Times the CPU oracle on the first n_tokens tokens of layer 0: routing,
+    then the SwiGLU experts and combine for those tokens.  Expert weights are
+    generated before the clock starts.  Returns (tokens/s, seconds, note)."""
+    from moe_inputs import device as mdev, gen
+    from oracle import workload as ow
+
+    li = gen.layer_inputs(cfg, 0)
+    toks = np.arange(min(n_tokens, cfg.T))
+    sub = gen.LayerInputs(x=li.x[toks], x_bits=None, wg=li.wg, bias=li.bias)
+    idx, w, _ = ow.route(cfg.with_(T=len(toks)), 0, sub)
+    pool, slot = mdev.default_placement(cfg)
+    cache = {}
+    pools = ow.split_pools(cfg, 0, pool, slot, cache)
+    for e in np.unique(idx):
+        pools.expert(int(e))  # generate (untimed)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        idx2, w2, _ = ow.route(cfg.with_(T=len(toks)), 0, sub)
+        ow.layer_tokens(cfg.with_(T=len(toks)), 0, np.arange(len(toks)), idx2, w2, pool, slot,
+                        sub, cache)
+    dt = time.perf_counter() - t0
+    return len(toks) * reps / dt, dt, f"first {len(toks)} token(s) of layer 0, {reps} pass(es)"
+
+
+def cpu_cores() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm.  One step is one ninth of one token's
+    MoE block: the token's routing (on its first step) and one of its k
+    routed experts or the shared expert, in fp64, accumulated into its output
+    row.  Tokens cycle over the first few of the workload; their expert
+    weights are generated before the clock starts."""
+    from moe_inputs import config, device as mdev, gen
+    from oracle import moe as om, workload as ow
+    cfg = config(args.config)
+    if rank != 0:
+        return None
+    parts = cfg.k + (1 if cfg.has_shared else 0)
+    n_tok = max(1, min(4, cfg.T, -(-(args.steps + args.warmup) // parts)))
+    li = gen.layer_inputs(cfg, 0)
+    pool, slot = mdev.default_placement(cfg)
+    cache = {}
+    pools = ow.split_pools(cfg, 0, pool, slot, cache)
+    sub_cfg = cfg.with_(T=1)
+    routes = []
+    for t in range(n_tok):
+        sub = gen.LayerInputs(x=li.x[t:t + 1], x_bits=None, wg=li.wg, bias=li.bias)
+        idx, w, _ = ow.route(sub_cfg, 0, sub)
+        routes.append((sub, idx, w))
+        for e in idx[0]:
+            pools.expert(int(e))          # generated before timing
+
+    def one_step(s):
+        t = (s // parts) % n_tok
+        part = s % parts
+        sub, idx, w = routes[t]
+        x64 = sub.x.astype(np.float64)
+        if part == 0:
+            ow.route(sub_cfg, 0, sub)
+        if part < cfg.k:
+            ex = pools.expert(int(idx[0, part]))
+            return w[0, part] * om.swiglu_ffn(x64, ex.gu_f64(), ex.down_f64())
+        return om.swiglu_ffn(x64, pools.shared.gu_f64(), pools.shared.down_f64())
+
+    for s in range(args.warmup):
+        one_step(s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        one_step(args.warmup + s)
+    dt = time.perf_counter() - t0
+    value = (args.steps / parts) / dt
+    note = (f"each step: 1/{parts} of one token's block on the CPU oracle (routing over all "
+            f"{cfg.E} experts on the token's first step, then one of its {cfg.k} routed experts "
+            f"or the shared expert, fp64); tokens cycle over the first {n_tok}")
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / max(args.steps, 1) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": workload_desc(cfg), "parallelism": "CPU oracle on rank 0"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "tokens/s", "cores": cpu_cores(),
+                         "kind": "oracle", "sample": note},
+        "e2e": {"value": round(value, 6), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------- main
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    out, cfg = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, note = oracle_sample(cfg, 6 if cfg.T > 64 else cfg.T)
+        out["cpu_baseline"] = {"value": round(v, 6), "unit": "tokens/s", "cores": cpu_cores(),
+                               "kind": "oracle", "sample": note + f" ({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -100,12 +100,22 @@ CONFIGS: dict[int, MoEConfig] = {
 }
 
 
+# Reduced cases of the same kernels for profiler captures, a few GB on the
+# device: the decode shape with 32 routed experts (about 4 tokens each, as in
+# the 128-token decode step) and the prefill shape with 32 experts.
+PROFILE_CASES: dict[int, MoEConfig] = {
+    21: CONFIGS[2].with_(cfg_id=21, name="r1_decode_shape_E32_T16", T=16, E=32, local_count=8),
+    23: CONFIGS[3].with_(cfg_id=23, name="r1_prefill_shape_E32_T1024", T=1024, E=32,
+                         local_count=8),
+}
+
+
 def config(cfg: int | str | MoEConfig) -> MoEConfig:
     if isinstance(cfg, MoEConfig):
         return cfg
     if isinstance(cfg, int):
-        return CONFIGS[cfg]
-    for c in CONFIGS.values():
+        return CONFIGS[cfg] if cfg in CONFIGS else PROFILE_CASES[cfg]
+    for c in list(CONFIGS.values()) + list(PROFILE_CASES.values()):
         if c.name == cfg:
             return c
     raise KeyError(cfg)
