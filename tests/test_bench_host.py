@@ -1,0 +1,76 @@
+"""bench.py's host-side plumbing on CPU: max/sum over ranks with gloo
+(world size 2), clock parsing, roofline arithmetic and argument defaults."""
+import os
+import socket
+
+import numpy as np
+import torch.multiprocessing as mp
+
+import bench
+from moe_inputs import config
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        mx = bench.max_over_ranks(10.0 + rank, world)
+        sm = bench.sum_over_ranks(128.0 * 3, world)
+        dist.barrier()
+        out[rank] = (mx, sm)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rank_reductions_with_gloo():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == out[1] == (11.0, 768.0)
+
+
+def test_single_rank_reductions_are_identity():
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.sum_over_ranks(7.0, 1) == 7.0
+
+
+def test_clock_summary_parsing():
+    c = bench.ClockSampler(0)
+    c.out = ("1935, 1965, Not Active, Not Active, Not Active, Active\n"
+             "1950, 1965, Not Active, Not Active, Not Active, Not Active\n"
+             "garbage\n")
+    s = c.summary()
+    assert s["sm_mhz"] == 1942.5 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 2
+
+
+def test_roofline_figures_decode_shape():
+    cfg = config(2)
+    counts = np.zeros(cfg.E, dtype=np.int64)
+    counts[:247] = 4
+    flops, nbytes = bench.roofline_figures(cfg, [counts], {})
+    per_expert = 3 * cfg.H * cfg.I * 2
+    assert nbytes == 248 * per_expert + 2 * cfg.T * cfg.H * 2
+    assert flops == (cfg.T * cfg.k + cfg.T) * 6 * cfg.H * cfg.I
+
+
+def test_default_arguments():
+    a = bench.parse_args([])
+    assert (a.gpus, a.config, a.impl) == (1, 2, "ours") and a.warmup >= 3
