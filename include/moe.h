@@ -147,6 +147,35 @@ MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const
                        float *x_perm_scales, void *workspace, size_t workspace_bytes,
                        cudaStream_t stream);
 
+/* Allocation-free moe_permute.  The DWDP pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory, not
+ * even a workspace of their own - for example a plug-in inside a host
+ * application or serving runtime that has reserved all device memory for its
+ * own pool and forbids any other allocation, or code on a latency-critical
+ * path where a cudaMalloc (which may synchronise the whole device) is not
+ * allowed.
+ *
+ * Same arguments and results as moe_permute without (workspace,
+ * workspace_bytes): the scratch lives in a fixed 1 MiB array inside the
+ * library's device memory, which every GPU that loads the library holds until
+ * the process exits.  It allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library call).
+ *   - Limit: moe_permute_workspace_size(T, k, E) <= 1 MiB, i.e.
+ *     8 * ceil(T*k / 2048) * E bytes (E = 256: up to 1,048,576 token-expert
+ *     assignments).  Larger sizes return MOE_ERR_WORKSPACE and enqueue nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (each word is written before it is
+ *     read within a call).  Calls that overlap on the GPU (other streams,
+ *     other host threads) race on it: serialise them. */
+MOE_API moe_status moe_permute_noalloc(int32_t T, int32_t k, int32_t E, int32_t H,
+                               const int32_t *topk_idx, const void *x, moe_dtype x_dtype,
+                               moe_dtype perm_dtype, int32_t with_shared, int32_t *offsets,
+                               int32_t *perm_src, int32_t *inv_pos, void *x_perm,
+                               float *x_perm_scales, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Expert weight images and the split-weight table.
  *

@@ -66,6 +66,8 @@ _SIGS = {
     "moe_permute_workspace_size": ([i32, i32, i32], sz),
     "moe_permute": ([i32, i32, i32, i32, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp],
                     i32),
+    "moe_permute_noalloc": ([i32, i32, i32, i32, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp],
+                           i32),
     "moe_expert_layout_get": ([i32, i32, i32, ctypes.POINTER(moe_expert_layout)], i32),
     "moe_grouped_ffn_workspace_size": ([ctypes.POINTER(moe_ffn_desc)], sz),
     "moe_grouped_ffn": ([ctypes.POINTER(moe_ffn_desc), ctypes.POINTER(moe_expert_table), vp, vp,
@@ -106,6 +108,7 @@ moe_route_workspace_size = _lib.moe_route_workspace_size
 moe_route = _lib.moe_route
 moe_permute_workspace_size = _lib.moe_permute_workspace_size
 moe_permute = _lib.moe_permute
+moe_permute_noalloc = _lib.moe_permute_noalloc
 moe_expert_layout_get = _lib.moe_expert_layout_get
 moe_grouped_ffn_workspace_size = _lib.moe_grouped_ffn_workspace_size
 moe_grouped_ffn = _lib.moe_grouped_ffn

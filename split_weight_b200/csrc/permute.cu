@@ -12,6 +12,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <mutex>
+
 #include "device.cuh"
 #include "internal.h"
 
@@ -309,6 +311,79 @@ moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t
         SWB_LAUNCHED("moe_permute: gather kernel");
     }
     return MOE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of moe_permute.
+//
+// For callers that cannot allocate device memory at all, not even a
+// workspace of their own: for example a plug-in running inside a host
+// application or serving runtime that has reserved all device memory for its
+// own pool and forbids any other allocation, or code on a latency-critical
+// path where a cudaMalloc (which may synchronise the whole device) is not
+// allowed.  The scratch that moe_permute takes as `workspace` (per-block
+// expert counts and bases) lives instead in a fixed array in this library's
+// device memory, created when the library is loaded and held by every GPU
+// that loads it until the process exits.
+// ---------------------------------------------------------------------------
+namespace swb {
+namespace {
+
+constexpr size_t kPermuteScratchBytes = size_t(1) << 20;  // 1 MiB per device
+static __device__ __align__(256) unsigned char g_permute_scratch[kPermuteScratchBytes];
+
+std::mutex g_scratch_mu;
+constexpr int kMaxScratchDevices = 64;
+void* g_scratch_addr[kMaxScratchDevices] = {nullptr};
+
+// Device address of g_permute_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device with cudaGetSymbolAddress (this is done by the first call
+// on each device) and cached.
+moe_status permute_scratch_address(void** out) {
+    int dev = 0;
+    SWB_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxScratchDevices)
+        return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: device %d", dev);
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cuda_injected_failure())
+            return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress: injected failure");
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
+        if (e != cudaSuccess) return cuda_check(e, "cudaGetSymbolAddress(permute scratch)");
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace swb
+
+extern "C" {
+
+moe_status moe_permute_noalloc(int32_t T, int32_t k, int32_t E, int32_t H,
+                               const int32_t* topk_idx, const void* x, moe_dtype x_dtype,
+                               moe_dtype perm_dtype, int32_t with_shared, int32_t* offsets,
+                               int32_t* perm_src, int32_t* inv_pos, void* x_perm,
+                               float* x_perm_scales, cudaStream_t stream) {
+    const size_t need = moe_permute_workspace_size(T, k, E);
+    if (need > kPermuteScratchBytes)
+        return fail(MOE_ERR_WORKSPACE,
+                    "moe_permute_noalloc: T=%d k=%d E=%d needs %zu bytes of scratch, more than "
+                    "the built-in %zu bytes (use moe_permute with a workspace)",
+                    T, k, E, need, kPermuteScratchBytes);
+    void* scratch = nullptr;
+    moe_status st = permute_scratch_address(&scratch);
+    if (st != MOE_OK) return st;
+    // Every scratch word the kernels read is written earlier in the same
+    // call (block counts, then bases), so nothing needs clearing first.
+    return moe_permute(T, k, E, H, topk_idx, x, x_dtype, perm_dtype, with_shared, offsets,
+                       perm_src, inv_pos, x_perm, x_perm_scales, scratch, kPermuteScratchBytes,
+                       stream);
 }
 
 }  // extern "C"
