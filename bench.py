@@ -222,22 +222,9 @@ def run_ours(args, rank, world, local_rank):
                 timed_ffn[0][1].record(stream)
             ml.combine(h)
             return
-        n = cfg.layers
-        for l, d in enumerate(dls):
-            ml = d.layer
-            ml.route(xs[l], h)
-            ml.permute(xs[l], h)
-            if prefetch:
-                stream.wait_event(pipe.ready[l])
-            if timed_ffn is not None:
-                timed_ffn[l][0].record(stream)
-            ml.grouped_ffn(h, pipe.bufs[l % 2])
-            if timed_ffn is not None:
-                timed_ffn[l][1].record(stream)
-            if prefetch:
-                pipe.free[l % 2].record(stream)
-                pipe._prefetch((l + 2) % n, pipe.free[l % 2])
-            ml.combine(h)
+        for l in range(cfg.layers):
+            pipe.run_layer(l, xs[l], stream, prefetch=prefetch,
+                           ffn_events=None if timed_ffn is None else timed_ffn[l])
 
     def barrier():
         if world > 1:
@@ -285,10 +272,11 @@ def run_ours(args, rank, world, local_rank):
         # copy alone
         c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         c0.record(pipe.copy_stream)
-        pipe._prefetch(0, None)
+        pipe.prefetch(0, 0, None)
         c1.record(pipe.copy_stream)
         torch.cuda.synchronize()
         copy_ms = c0.elapsed_time(c1)
+        pipe.g = 0
         pipe.prime()
         torch.cuda.synchronize()
         piped_ms = elapsed_ms / args.steps

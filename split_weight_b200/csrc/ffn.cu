@@ -11,13 +11,19 @@
 // One persistent, warp-specialised kernel per GEMM (sm_100a):
 //   warp 0      TMA producer (one thread): weight tile(s) + token rows
 //   warp 1      tcgen05.mma issuer (one thread); owns the TMEM allocation
-//   warps 2-5   epilogue: TMEM -> registers -> (SwiGLU) -> bf16 -> global
-// The MMA puts the weight rows on M (128) and the expert's tokens on N
-// (16..BN), so a decode-sized expert with 4 tokens costs an N=16 MMA, not a
-// 128-row tile.  GEMM1 keeps two fp32 accumulators per tile, gate and up for
-// the same 128 features, so SwiGLU is fused in the epilogue.  Accumulators
-// are double buffered in TMEM so the epilogue of one tile overlaps the next
-// tile's main loop.
+//   warps 2..   epilogue (4 or 8 warps): TMEM -> registers -> (SwiGLU) -> bf16
+// The MMA puts weight rows on M (128 per instruction) and the expert's tokens
+// on N (16..256), so a decode-sized expert with 4 tokens costs an N=16 MMA,
+// not a 128-row tile.  A CTA holds one or two weight tiles per stage:
+//   GATED  gate rows and up rows of the same 128 features, two fp32
+//          accumulators, SwiGLU fused in the epilogue (GEMM1);
+//   PAIR   two adjacent 128-row blocks (256 output features, GEMM2);
+//   SINGLE one 128-row block.
+// Both weight tiles share the token tile, which halves the activation bytes
+// each MMA needs.  Accumulators are double buffered in TMEM when they fit
+// (two buffers of up to 256 columns) so the epilogue of one tile overlaps
+// the next tile's main loop; the widest tiles (2 x 256 columns) use all 512
+// TMEM columns in one buffer and 8 epilogue warps.
 #include <cuda_bf16.h>
 
 #include "device.cuh"
@@ -31,7 +37,6 @@ constexpr int kBM = 128;                       // weight rows per tile (MMA M)
 constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle atom
 constexpr int kBoxN = 16;                      // token rows per TMA box
 constexpr uint32_t kABytes = kBM * kBK * 2;    // one weight tile, 16 KB
-constexpr int kThreads = 192;
 constexpr uint32_t kSmemBudget = 200 * 1024;   // pipeline stages
 
 struct alignas(64) FfnArgs {
@@ -48,14 +53,23 @@ struct alignas(64) FfnArgs {
     int32_t pool_slot[kMaxGroups];  // (pool << 31) | slot per routed expert
 };
 
-template <int BN, bool GATED>
+enum { kSingle = 0, kGated = 1, kPair = 2 };
+
+template <int BN, int MODE>
 struct Cfg {
-    static constexpr uint32_t kAStage = kABytes * (GATED ? 2 : 1);
+    static constexpr int kNA = MODE == kSingle ? 1 : 2;           // weight tiles per stage
+    static constexpr uint32_t kAStage = kABytes * kNA;
     static constexpr uint32_t kStageBytes = kAStage + BN * kBK * 2;
     static constexpr int kStages = (kSmemBudget / kStageBytes) > 12 ? 12 : (kSmemBudget / kStageBytes);
-    static constexpr uint32_t kAccCols = (GATED ? 2 : 1) * BN;
-    static constexpr uint32_t kTmemCols = 2 * kAccCols;
+    static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
+    static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+    static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
+    static constexpr int kEpiWarps = BN >= 256 ? 8 : 4;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    static constexpr int kRowsPerTile = MODE == kPair ? 2 * kBM : kBM;  // output features
     static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024;
+    static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                  "TMEM allocation must be a power of two in [32, 512]");
 };
 
 struct Tile {
@@ -69,8 +83,8 @@ struct Tables {
     int ps[kMaxGroups];  // (map << 24) | slot   (map 0 local, 1 remote, 2 shared)
 };
 
-template <int BN>
-__device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G, int MT) {
+template <int BN, int ROWS>
+__device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
     int lo = 0, hi = G - 1;
     while (lo < hi) {  // largest group whose first tile is <= tile (never an empty one)
         const int mid = (lo + hi + 1) >> 1;
@@ -81,21 +95,21 @@ __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G, i
     const int ntn = (n + BN - 1) / BN;
     const int mt = local / ntn, nt = local - mt * ntn;
     Tile t;
-    t.m0 = mt * kBM;
+    t.m0 = mt * ROWS;
     t.row0 = tb.row0[g] + nt * BN;
     t.n_rows = min(BN, n - nt * BN);
     t.n_mma = (t.n_rows + 15) & ~15;
     t.map = tb.ps[g] >> 24;
     t.slot = tb.ps[g] & 0xFFFFFF;
-    (void)MT;
     return t;
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-template <int BN, bool GATED>
-__global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_constant__ FfnArgs p) {
-    using C = Cfg<BN, GATED>;
+template <int BN, int MODE>
+__global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
+    k_grouped_ffn(const __grid_constant__ FfnArgs p) {
+    using C = Cfg<BN, MODE>;
     extern __shared__ uint8_t dyn_smem[];
     __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
@@ -106,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t stages = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     const int G = p.E + (p.has_shared ? 1 : 0);
-    const int MT = p.M / kBM;
+    const int MT = p.M / C::kRowsPerTile;
     const int KB = p.K / kBK;
     volatile int* abort_flag = &abort_sh;
 
@@ -118,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&acc_full[a]), 1);
-            mbar_init(smem_u32(&acc_empty[a]), 4);
+            mbar_init(smem_u32(&acc_empty[a]), C::kEpiWarps);
         }
         fence_mbar_init();
         tma_prefetch_map(&p.act_map);
@@ -175,9 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile<BN>(tile, tb, G, MT);
+                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
                 const CUtensorMap* wm = &p.w_map[t.map];
                 const uint32_t tx = C::kAStage + (uint32_t)t.n_mma * kBK * 2;
+                const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
                 for (int kb = 0; kb < KB; ++kb) {
                     const uint32_t eb = smem_u32(&empty_bar[stage]);
                     const uint32_t fb = smem_u32(&full_bar[stage]);
@@ -188,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
                     const uint32_t sa = stages + stage * C::kStageBytes;
                     mbar_arrive_expect_tx(fb, tx);
                     tma_load_3d(sa, wm, fb, kb * kBK, t.m0, t.slot);
-                    if constexpr (GATED) tma_load_3d(sa + kABytes, wm, fb, kb * kBK, p.up_row + t.m0, t.slot);
+                    if constexpr (C::kNA == 2) tma_load_3d(sa + kABytes, wm, fb, kb * kBK, row_a1, t.slot);
                     const uint32_t sb = sa + C::kAStage;
                     for (int i = 0; i < t.n_mma / kBoxN; ++i)
                         tma_load_2d(sb + i * kBoxN * kBK * 2, &p.act_map, fb, kb * kBK,
@@ -207,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
             uint32_t phase = 0, acc_use[2] = {0u, 0u};
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile<BN>(tile, tb, G, MT);
+                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
                 if (!mbar_wait(smem_u32(&acc_empty[acc]), (acc_use[acc] & 1u) ^ 1u, abort_flag,
                                p.err))
                     break;
@@ -227,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
                         const uint32_t accum = (kb | kk) != 0;
                         const uint64_t bd = sw128_desc(sb + kk * 32);
                         mma_bf16_ss(d0, sw128_desc(sa + kk * 32), bd, idesc, accum);
-                        if constexpr (GATED)
+                        if constexpr (C::kNA == 2)
                             mma_bf16_ss(d0 + BN, sw128_desc(sa + kABytes + kk * 32), bd, idesc, accum);
                     }
                     mma_commit(smem_u32(&empty_bar[stage]));
@@ -239,33 +254,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
                 if (!ok) break;
                 mma_commit(smem_u32(&acc_full[acc]));
                 ++acc_use[acc];
-                acc ^= 1;
+                if (C::kAccBufs == 2) acc ^= 1;
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 2..5)
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;                    // TMEM lane quarter this warp may access
+        const int part = (warp - 2) >> 2;          // column half (8 epilogue warps) or 0
+        constexpr int kCols = C::kEpiWarps == 8 ? BN / 2 : BN;
         int acc = 0;
         uint32_t acc_use[2] = {0u, 0u};
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile<BN>(tile, tb, G, MT);
+            const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
             bool ok = mbar_wait(smem_u32(&acc_full[acc]), acc_use[acc] & 1u, abort_flag, p.err);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::kAccCols;
             const int f = t.m0 + 32 * q + lane;
             __nv_bfloat16* out = p.out + (int64_t)t.row0 * p.ld_out + f;
-            for (int c0 = 0; c0 < t.n_rows; c0 += 16) {
+            const int c_begin = part * kCols, c_end = min(t.n_rows, c_begin + kCols);
+            for (int c0 = c_begin; c0 < c_end; c0 += 16) {
                 float g[16];
                 tmem_ld_16(tacc + c0, g);
-                if constexpr (GATED) {
+                if constexpr (C::kNA == 2) {
                     float u[16];
                     tmem_ld_16(tacc + BN + c0, u);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c0 + i < t.n_rows)
-                            out[(int64_t)(c0 + i) * p.ld_out] = __float2bfloat16_rn(silu_mul(g[i], u[i]));
+                    for (int i = 0; i < 16; ++i) {
+                        if (c0 + i >= t.n_rows) continue;
+                        __nv_bfloat16* o = out + (int64_t)(c0 + i) * p.ld_out;
+                        if constexpr (MODE == kGated) {
+                            o[0] = __float2bfloat16_rn(silu_mul(g[i], u[i]));
+                        } else {
+                            o[0] = __float2bfloat16_rn(g[i]);
+                            o[kBM] = __float2bfloat16_rn(u[i]);
+                        }
+                    }
                 } else {
                     tmem_ld_wait();
 #pragma unroll
@@ -278,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
             ++acc_use[acc];
-            acc ^= 1;
+            if (C::kAccBufs == 2) acc ^= 1;
         }
     }
 
@@ -295,41 +320,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_grouped_ffn(const __grid_consta
 }
 
 // ---------------------------------------------------------------- host side
-template <int BN, bool GATED>
+template <int BN, int MODE>
 moe_status launch(const FfnArgs& a, int rows, int G, cudaStream_t s) {
-    using C = Cfg<BN, GATED>;
+    using C = Cfg<BN, MODE>;
     int sms = 0;
     moe_status st = sm_count(&sms);
     if (st != MOE_OK) return st;
-    const int64_t mt = a.M / kBM;
+    const int64_t mt = a.M / C::kRowsPerTile;
     const int64_t bound = mt * ((rows + BN - 1) / BN + G);
     const int grid = (int)(bound < sms ? bound : sms);
     if (grid <= 0) return MOE_OK;
-    auto kern = k_grouped_ffn<BN, GATED>;
+    auto kern = k_grouped_ffn<BN, MODE>;
     SWB_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)C::kDynSmem));
-    kern<<<grid, kThreads, C::kDynSmem, s>>>(a);
-    SWB_LAUNCHED(GATED ? "moe_grouped_ffn: gate/up kernel" : "moe_grouped_ffn: down kernel");
+    kern<<<grid, C::kThreads, C::kDynSmem, s>>>(a);
+    SWB_LAUNCHED(MODE == kGated ? "moe_grouped_ffn: gate/up kernel" : "moe_grouped_ffn: down kernel");
     return MOE_OK;
 }
 
-template <bool GATED>
+template <int MODE>
 moe_status launch_bn(int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) {
     switch (bn) {
-        case 16: return launch<16, GATED>(a, rows, G, s);
-        case 32: return launch<32, GATED>(a, rows, G, s);
-        case 64: return launch<64, GATED>(a, rows, G, s);
-        default: return launch<128, GATED>(a, rows, G, s);
+        case 16: return launch<16, MODE>(a, rows, G, s);
+        case 32: return launch<32, MODE>(a, rows, G, s);
+        case 64: return launch<64, MODE>(a, rows, G, s);
+        case 128: return launch<128, MODE>(a, rows, G, s);
+        default: return launch<256, MODE>(a, rows, G, s);
     }
 }
 
-// Token tile: about twice the mean tokens per expert, 16..128.
+// Token tile from the mean tokens per routed expert, 16..256.
 int pick_bn(int64_t A, int E) {
     const int64_t mean = (A + E - 1) / E;
     if (mean <= 8) return 16;
     if (mean <= 16) return 32;
     if (mean <= 32) return 64;
-    return 128;
+    if (mean <= 160) return 128;
+    return 256;
 }
 
 moe_status encode_weight_map(CUtensorMap* m, const void* base, int64_t offset, int32_t count,
@@ -452,7 +479,7 @@ moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, c
     a.up_row = d->I;
     a.out = static_cast<__nv_bfloat16*>(h);
     a.ld_out = d->I;
-    if ((st = launch_bn<true>(bn, a, (int)rows, G, stream)) != MOE_OK) return st;
+    if ((st = launch_bn<kGated>(bn, a, (int)rows, G, stream)) != MOE_OK) return st;
 
     // GEMM2: y = h W_down^T
     for (int q = 0; q < 2; ++q)
@@ -468,7 +495,8 @@ moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, c
     a.up_row = 0;
     a.out = static_cast<__nv_bfloat16*>(y_perm);
     a.ld_out = d->H;
-    return launch_bn<false>(bn, a, (int)rows, G, stream);
+    if (d->H % (2 * kBM) == 0) return launch_bn<kPair>(bn, a, (int)rows, G, stream);
+    return launch_bn<kSingle>(bn, a, (int)rows, G, stream);
 }
 
 }  // extern "C"

@@ -193,10 +193,14 @@ class PrefetchPipeline:
     """Consecutive MoE layers whose remote experts are fetched ahead into two
     alternate buffers by moe_prefetch_layer on a copy-engine stream.
 
-    Layer l computes from remote_bufs[l % 2]; as soon as layer l's grouped
-    GEMMs have been enqueued, the copy stream waits for them (free event) and
-    starts fetching layer l + 2 into the same buffer.  Layer l waits for its
-    own ready event before its grouped GEMM.
+    Layer executions are numbered g = 0, 1, 2, ... across passes; execution g
+    computes from bufs[g % 2].  As soon as its grouped GEMMs are enqueued,
+    the compute stream records free[g % 2] and the copy stream, after waiting
+    for it, fetches the layer of execution g + 2 into the same buffer and
+    records ready[g % 2], which execution g + 2 waits for before its grouped
+    GEMM.  With wrap=True the fetches issued by the last layers of a pass are
+    those of the next pass's first layers, as in a steady stream of forward
+    passes.
     """
 
     def __init__(self, layers: list[MoELayer], peer_stores: list[torch.Tensor],
@@ -205,43 +209,54 @@ class PrefetchPipeline:
         self.remote_bytes, self.chunk_bytes = remote_bytes, chunk_bytes
         dev = torch.device(device)
         self.bufs = [torch.empty(max(remote_bytes, 1), dtype=torch.uint8, device=dev)
-                     for _ in range(min(2, len(layers)))]
+                     for _ in range(2)]
         self.copy_stream = torch.cuda.Stream(device=dev)
-        self.ready = [torch.cuda.Event() for _ in layers]
-        self.free = [torch.cuda.Event() for _ in self.bufs]
+        self.ready = [torch.cuda.Event() for _ in range(2)]
+        self.free = [torch.cuda.Event() for _ in range(2)]
+        for ev in self.ready + self.free:   # torch creates CUDA events on first record
+            ev.record(self.copy_stream)
+        self.g = 0
 
-    def _prefetch(self, l: int, wait_free: torch.cuda.Event | None) -> None:
-        L.check(L.moe_prefetch_layer(self.peer_stores[l].data_ptr(), self.bufs[l % 2].data_ptr(),
+    def prefetch(self, layer: int, buf: int, wait_free: torch.cuda.Event | None) -> None:
+        assert self.ready[buf].cuda_event != 0 and (wait_free is None or wait_free.cuda_event != 0)
+        L.check(L.moe_prefetch_layer(self.peer_stores[layer].data_ptr(), self.bufs[buf].data_ptr(),
                                      self.remote_bytes, self.chunk_bytes,
                                      self.copy_stream.cuda_stream,
                                      wait_free.cuda_event if wait_free is not None else None,
-                                     self.ready[l].cuda_event))
+                                     self.ready[buf].cuda_event))
 
     def prime(self) -> None:
-        """Enqueues the fetch of the first two layers (before the timed loop)."""
-        for l in range(len(self.bufs)):
-            self._prefetch(l, None)
+        """Enqueues the fetches of the next two executions (before a run)."""
+        n = len(self.layers)
+        for i in range(2):
+            self.prefetch((self.g + i) % n, (self.g + i) % 2, None)
+
+    def run_layer(self, l: int, x: torch.Tensor, stream: torch.cuda.Stream,
+                  prefetch: bool = True, wrap: bool = True, ffn_events=None) -> torch.Tensor:
+        """One layer execution; ffn_events = (start, end) events around its
+        grouped GEMMs, if given."""
+        n = len(self.layers)
+        layer, h, b = self.layers[l], stream.cuda_stream, self.g % 2
+        layer.route(x, h)
+        layer.permute(x, h)
+        if prefetch:
+            stream.wait_event(self.ready[b])
+        if ffn_events is not None:
+            ffn_events[0].record(stream)
+        layer.grouped_ffn(h, self.bufs[b])
+        if ffn_events is not None:
+            ffn_events[1].record(stream)
+        if prefetch and (l + 2 < n or wrap):
+            self.free[b].record(stream)
+            self.prefetch((l + 2) % n, b, self.free[b])
+        layer.combine(h)
+        self.g += 1
+        return layer.y
 
     def run(self, xs: list[torch.Tensor], stream: torch.cuda.Stream | None = None,
             prefetch: bool = True, wrap: bool = True) -> list[torch.Tensor]:
-        """Runs all layers.  With prefetch=False the buffers are used as they
-        are (nothing is copied).  With wrap=True the fetches issued during the
-        last layers are those of the next pass's first layers, as in a
-        steady stream of forward passes; prime() must have run once."""
+        """Runs all layers once.  With prefetch=False nothing is copied and
+        the buffers are used as they are; prime() must have run once before
+        the first pass with prefetch."""
         stream = stream if stream is not None else torch.cuda.current_stream()
-        h = stream.cuda_stream
-        outs = []
-        n = len(self.layers)
-        for l, layer in enumerate(self.layers):
-            layer.route(xs[l], h)
-            layer.permute(xs[l], h)
-            if prefetch:
-                stream.wait_event(self.ready[l])
-            layer.grouped_ffn(h, self.bufs[l % 2])
-            nxt = l + 2
-            if prefetch and (nxt < n or (wrap and n >= 2)):
-                self.free[l % 2].record(stream)
-                self._prefetch(nxt % n, self.free[l % 2])
-            layer.combine(h)
-            outs.append(layer.y)
-        return outs
+        return [self.run_layer(l, xs[l], stream, prefetch, wrap) for l in range(len(self.layers))]
