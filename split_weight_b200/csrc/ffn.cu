@@ -25,6 +25,8 @@
 // the next tile's main loop; the widest tiles (2 x 256 columns) use all 512
 // TMEM columns in one buffer and 8 epilogue warps.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "device.cuh"
 #include "internal.h"
@@ -41,7 +43,8 @@ constexpr uint32_t kSmemBudget = 200 * 1024;   // pipeline stages
 
 struct alignas(64) FfnArgs {
     CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}
-    CUtensorMap act_map;       // activation rows {K, rows}
+    CUtensorMap act_map;       // activation rows {K, rows}, 16-row box
+    CUtensorMap act_map64;     // the same rows, 64-row box
     const int32_t* offsets;    // [E+1] first row of each expert
     __nv_bfloat16* out;        // [rows, ld_out]
     int* err;                  // device error word
@@ -51,25 +54,41 @@ struct alignas(64) FfnArgs {
     int32_t up_row;            // GEMM1: first row of the "up" half of w_gu (= I)
     int32_t ld_out;
     int32_t pool_slot[kMaxGroups];  // (pool << 31) | slot per routed expert
+    // e4m3 weights only: block scales of (slot, row block, k block) at
+    // w_base[map] + slot * w_stride[map] + scale_off + 4 * (row_block * kblocks + k_block)
+    const uint8_t* w_base[3];
+    int64_t w_stride[3];
+    int64_t scale_off;
+    int32_t kblocks;
 };
 
 enum { kSingle = 0, kGated = 1, kPair = 2 };
 
-template <int BN, int MODE>
+constexpr uint32_t kA8Bytes = kBM * kBK;       // one e4m3 weight tile as loaded, 8 KB
+constexpr int kConvThreads = 128;              // e4m3 -> bf16 converter warps (4)
+
+// Per stage: the bf16 weight tile(s) the MMA reads (128-byte swizzled), the
+// token tile, and for e4m3 weights the staging tile(s) TMA writes.
+template <int BN, int MODE, bool W8>
 struct Cfg {
     static constexpr int kNA = MODE == kSingle ? 1 : 2;           // weight tiles per stage
     static constexpr uint32_t kAStage = kABytes * kNA;
-    static constexpr uint32_t kStageBytes = kAStage + BN * kBK * 2;
+    static constexpr uint32_t kBStage = BN * kBK * 2;
+    static constexpr uint32_t kA8Stage = W8 ? kA8Bytes * kNA : 0;
+    static constexpr uint32_t kStageBytes = kAStage + kBStage + kA8Stage;
     static constexpr int kStages = (kSmemBudget / kStageBytes) > 12 ? 12 : (kSmemBudget / kStageBytes);
     static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
     static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
     static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
     static constexpr int kEpiWarps = BN >= 256 ? 8 : 4;
-    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    static constexpr int kConvWarps = W8 ? kConvThreads / 32 : 0;
+    static constexpr int kConvFirstWarp = 2 + kEpiWarps;
+    static constexpr int kThreads = 64 + 32 * (kEpiWarps + kConvWarps);
     static constexpr int kRowsPerTile = MODE == kPair ? 2 * kBM : kBM;  // output features
     static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024;
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                   "TMEM allocation must be a power of two in [32, 512]");
+    static_assert(kStages >= 2, "pipeline needs two stages");
 };
 
 struct Tile {
@@ -83,6 +102,23 @@ struct Tables {
     int ps[kMaxGroups];  // (map << 24) | slot   (map 0 local, 1 remote, 2 shared)
 };
 
+// An expert's n rows are cut into equal token tiles of tr rows (a multiple of
+// 16, at most BN): tiles of one expert that stream the same weights then run
+// at the same pace, so the second one finds the weights still in L2.
+template <int BN>
+__device__ __host__ __forceinline__ int tile_rows(int n) {
+    const int ntn = (n + BN - 1) / BN;
+    const int per = (n + ntn - 1) / ntn;
+    return (per + 15) & ~15;
+}
+
+template <int BN>
+__device__ __host__ __forceinline__ int token_tiles(int n) {
+    if (n <= 0) return 0;
+    const int tr = tile_rows<BN>(n);
+    return (n + tr - 1) / tr;
+}
+
 template <int BN, int ROWS>
 __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
     int lo = 0, hi = G - 1;
@@ -92,12 +128,13 @@ __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
         else hi = mid - 1;
     }
     const int g = lo, local = tile - tb.tile_start[g], n = tb.n[g];
-    const int ntn = (n + BN - 1) / BN;
+    const int tr = tile_rows<BN>(n);
+    const int ntn = (n + tr - 1) / tr;
     const int mt = local / ntn, nt = local - mt * ntn;
     Tile t;
     t.m0 = mt * ROWS;
-    t.row0 = tb.row0[g] + nt * BN;
-    t.n_rows = min(BN, n - nt * BN);
+    t.row0 = tb.row0[g] + nt * tr;
+    t.n_rows = min(tr, n - nt * tr);
     t.n_mma = (t.n_rows + 15) & ~15;
     t.map = tb.ps[g] >> 24;
     t.slot = tb.ps[g] & 0xFFFFFF;
@@ -106,12 +143,33 @@ __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-template <int BN, int MODE>
-__global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
+// 16 e4m3 weights (one 16-byte chunk of a staged row) times their block
+// scale, rounded to bf16: 32 bytes, the two 16-byte chunks that follow.
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 in, float s, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * h));
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * s, f.y * s);
+            o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int BN, int MODE, bool W8>
+__global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     k_grouped_ffn(const __grid_constant__ FfnArgs p) {
-    using C = Cfg<BN, MODE>;
+    using C = Cfg<BN, MODE, W8>;
     extern __shared__ uint8_t dyn_smem[];
     __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
+    __shared__ __align__(8) uint64_t conv_bar[W8 ? C::kStages : 1];  // bf16 tiles converted
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -129,6 +187,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&empty_bar[s]), 1);
+            if constexpr (W8) mbar_init(smem_u32(&conv_bar[s]), C::kConvWarps);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&acc_full[a]), 1);
@@ -136,6 +195,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
         }
         fence_mbar_init();
         tma_prefetch_map(&p.act_map);
+        tma_prefetch_map(&p.act_map64);
         for (int m = 0; m < 3; ++m) tma_prefetch_map(&p.w_map[m]);
     }
     if (warp == 1) {
@@ -161,7 +221,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
             tb.row0[g] = r0;
             tb.n[g] = n;
             tb.ps[g] = ps;
-            sum += ((n + BN - 1) / BN) * MT;
+            sum += token_tiles<BN>(n) * MT;
         }
         int incl = sum;
 #pragma unroll
@@ -172,7 +232,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
         int run = incl - sum;
         for (int g = g0; g < g1; ++g) {
             tb.tile_start[g] = run;
-            run += ((tb.n[g] + BN - 1) / BN) * MT;
+            run += token_tiles<BN>(tb.n[g]) * MT;
         }
         if (lane == 31) tb.tile_start[G] = incl;
     }
@@ -191,7 +251,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
                 const CUtensorMap* wm = &p.w_map[t.map];
-                const uint32_t tx = C::kAStage + (uint32_t)t.n_mma * kBK * 2;
+                const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
                 const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
                 for (int kb = 0; kb < KB; ++kb) {
                     const uint32_t eb = smem_u32(&empty_bar[stage]);
@@ -202,12 +262,17 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
                     }
                     const uint32_t sa = stages + stage * C::kStageBytes;
                     mbar_arrive_expect_tx(fb, tx);
-                    tma_load_3d(sa, wm, fb, kb * kBK, t.m0, t.slot);
-                    if constexpr (C::kNA == 2) tma_load_3d(sa + kABytes, wm, fb, kb * kBK, row_a1, t.slot);
+                    // e4m3 weights land in the staging area, bf16 ones straight in the operand
+                    const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
+                    const uint32_t w_step = W8 ? kA8Bytes : kABytes;
+                    tma_load_3d(sw, wm, fb, kb * kBK, t.m0, t.slot);
+                    if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * kBK, row_a1, t.slot);
                     const uint32_t sb = sa + C::kAStage;
-                    for (int i = 0; i < t.n_mma / kBoxN; ++i)
-                        tma_load_2d(sb + i * kBoxN * kBK * 2, &p.act_map, fb, kb * kBK,
-                                    t.row0 + i * kBoxN);
+                    int r = 0;
+                    for (; r + 64 <= t.n_mma; r += 64)
+                        tma_load_2d(sb + r * kBK * 2, &p.act_map64, fb, kb * kBK, t.row0 + r);
+                    for (; r < t.n_mma; r += kBoxN)
+                        tma_load_2d(sb + r * kBK * 2, &p.act_map, fb, kb * kBK, t.row0 + r);
                     if (++stage == C::kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -230,7 +295,8 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
                 const uint32_t idesc = idesc_bf16_f32(kBM, t.n_mma);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err)) {
+                    const uint32_t ready_bar = W8 ? smem_u32(&conv_bar[stage]) : smem_u32(&full_bar[stage]);
+                    if (!mbar_wait(ready_bar, phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
@@ -255,6 +321,63 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
                 mma_commit(smem_u32(&acc_full[acc]));
                 ++acc_use[acc];
                 if (C::kAccBufs == 2) acc ^= 1;
+            }
+        }
+    } else if (W8 && warp >= C::kConvFirstWarp) {
+        // ------------------------------------------------ e4m3 -> bf16 converters
+        // Each staged row is 64 e4m3 bytes (4 chunks of 16); the bf16 operand
+        // row is 128 bytes in the 128-byte swizzle: 16-byte chunk j of row r
+        // sits at position j ^ (r % 8).  One 128x128 block scale covers the
+        // whole stage (64 columns of K, 128 rows).
+        const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. 127
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+            const uint8_t* sbase = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map] + p.scale_off;
+            const float* sc0 = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
+            const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
+            const float* sc1 = reinterpret_cast<const float*>(sbase) + (int64_t)rb1 * p.kblocks;
+            for (int kb = 0; kb < KB; ++kb) {
+                const float s0 = __ldg(sc0 + (kb >> 1));
+                const float s1 = C::kNA == 2 ? __ldg(sc1 + (kb >> 1)) : 0.0f;
+                ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = stages + stage * C::kStageBytes;
+                const uint32_t s8 = sa + C::kAStage + C::kBStage;
+#pragma unroll
+                for (int a = 0; a < C::kNA; ++a) {
+                    const float sc = a == 0 ? s0 : s1;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int id = ct + kConvThreads * i, r = id >> 2, c = id & 3;
+                        uint4 in, lo, hi;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(in.x), "=r"(in.y), "=r"(in.z), "=r"(in.w)
+                                     : "r"(s8 + a * kA8Bytes + r * kBK + c * 16));
+                        e4m3x16_to_bf16(in, sc, lo, hi);
+                        const uint32_t row = sa + a * kABytes + r * 128;
+                        const uint32_t j0 = (2 * c) ^ (r & 7), j1 = (2 * c + 1) ^ (r & 7);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j0 * 16),
+                                     "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
+                                     : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j1 * 16),
+                                     "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                                     : "memory");
+                    }
+                }
+                // generic-proxy stores -> visible to the tensor core's async proxy
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&conv_bar[stage]));
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
     } else {
@@ -320,17 +443,17 @@ __global__ void __launch_bounds__(Cfg<BN, MODE>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-template <int BN, int MODE>
+template <int BN, int MODE, bool W8>
 moe_status launch(const FfnArgs& a, int rows, int G, cudaStream_t s) {
-    using C = Cfg<BN, MODE>;
+    using C = Cfg<BN, MODE, W8>;
     int sms = 0;
     moe_status st = sm_count(&sms);
     if (st != MOE_OK) return st;
     const int64_t mt = a.M / C::kRowsPerTile;
-    const int64_t bound = mt * ((rows + BN - 1) / BN + G);
+    const int64_t bound = mt * ((rows + 15) / 16 + G);
     const int grid = (int)(bound < sms ? bound : sms);
     if (grid <= 0) return MOE_OK;
-    auto kern = k_grouped_ffn<BN, MODE>;
+    auto kern = k_grouped_ffn<BN, MODE, W8>;
     SWB_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)C::kDynSmem));
     kern<<<grid, C::kThreads, C::kDynSmem, s>>>(a);
@@ -338,15 +461,20 @@ moe_status launch(const FfnArgs& a, int rows, int G, cudaStream_t s) {
     return MOE_OK;
 }
 
-template <int MODE>
+template <int MODE, bool W8>
 moe_status launch_bn(int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) {
     switch (bn) {
-        case 16: return launch<16, MODE>(a, rows, G, s);
-        case 32: return launch<32, MODE>(a, rows, G, s);
-        case 64: return launch<64, MODE>(a, rows, G, s);
-        case 128: return launch<128, MODE>(a, rows, G, s);
-        default: return launch<256, MODE>(a, rows, G, s);
+        case 16: return launch<16, MODE, W8>(a, rows, G, s);
+        case 32: return launch<32, MODE, W8>(a, rows, G, s);
+        case 64: return launch<64, MODE, W8>(a, rows, G, s);
+        case 128: return launch<128, MODE, W8>(a, rows, G, s);
+        default: return launch<256, MODE, W8>(a, rows, G, s);
     }
+}
+
+template <int MODE>
+moe_status launch_w(bool w8, int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) {
+    return w8 ? launch_bn<MODE, true>(bn, a, rows, G, s) : launch_bn<MODE, false>(bn, a, rows, G, s);
 }
 
 // Token tile from the mean tokens per routed expert, 16..256.
@@ -359,20 +487,24 @@ int pick_bn(int64_t A, int E) {
     return 256;
 }
 
+// 3-D map {K, rows, slot} over one pool of expert images.  bf16 weights are
+// loaded straight into the MMA operand layout (128-byte swizzle); e4m3
+// weights as plain 64-byte rows for the converter warps.
 moe_status encode_weight_map(CUtensorMap* m, const void* base, int64_t offset, int32_t count,
-                             int64_t stride, int32_t K, int32_t rows) {
+                             int64_t stride, int32_t K, int32_t rows, bool w8) {
     const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)count};
-    const uint64_t strides[2] = {(uint64_t)K * 2, (uint64_t)stride};
+    const uint64_t strides[2] = {(uint64_t)K * (w8 ? 1 : 2), (uint64_t)stride};
     const uint32_t box[3] = {(uint32_t)kBK, (uint32_t)kBM, 1u};
-    return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    return encode_tiled(m, w8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                         const_cast<char*>(static_cast<const char*>(base)) + offset, dims, strides,
-                        box, CU_TENSOR_MAP_SWIZZLE_128B);
+                        box, w8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-moe_status encode_act_map(CUtensorMap* m, const void* base, int64_t rows, int32_t K) {
+moe_status encode_act_map(CUtensorMap* m, const void* base, int64_t rows, int32_t K,
+                          uint32_t box_rows) {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
     const uint64_t strides[1] = {(uint64_t)K * 2};
-    const uint32_t box[2] = {(uint32_t)kBK, (uint32_t)kBoxN};
+    const uint32_t box[2] = {(uint32_t)kBK, box_rows};
     return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
@@ -383,7 +515,7 @@ moe_status validate(const moe_ffn_desc* d, const moe_expert_table* tb, moe_exper
         d->H <= 0 || d->I <= 0 || d->H % 128 || d->I % 128)
         return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: T=%d H=%d I=%d E=%d k=%d", d->T, d->H,
                     d->I, d->E, d->k);
-    if (d->w_dtype != MOE_BF16 || d->act_dtype != MOE_BF16)
+    if ((d->w_dtype != MOE_BF16 && d->w_dtype != MOE_E4M3) || d->act_dtype != MOE_BF16)
         return fail(MOE_ERR_UNSUPPORTED, "moe_grouped_ffn: weight dtype %d / activation dtype %d",
                     d->w_dtype, d->act_dtype);
     moe_status st = moe_expert_layout_get(d->H, d->I, (moe_dtype)d->w_dtype, lay);
@@ -464,39 +596,52 @@ moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, c
     const int32_t count[2] = {tbl->local_count, tbl->remote_count};
     const int64_t stride[2] = {tbl->local_stride, tbl->remote_stride};
     const int bn = pick_bn(A, d->E);
+    const bool w8 = d->w_dtype == MOE_E4M3;
+    a.w_base[0] = static_cast<const uint8_t*>(tbl->local_base);
+    a.w_base[1] = static_cast<const uint8_t*>(tbl->remote_base);
+    a.w_base[2] = static_cast<const uint8_t*>(tbl->shared);
+    a.w_stride[0] = tbl->local_stride;
+    a.w_stride[1] = tbl->remote_stride;
+    a.w_stride[2] = lay.bytes;
 
     // GEMM1: h = silu(X W_gate^T) * (X W_up^T)
     for (int q = 0; q < 2; ++q)
         if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.gu_offset, count[q],
-                                                    stride[q], d->H, 2 * d->I)) != MOE_OK)
+                                                    stride[q], d->H, 2 * d->I, w8)) != MOE_OK)
             return st;
     if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.gu_offset, 1,
-                                                 lay.bytes, d->H, 2 * d->I)) != MOE_OK)
+                                                 lay.bytes, d->H, 2 * d->I, w8)) != MOE_OK)
         return st;
-    if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H)) != MOE_OK) return st;
+    a.scale_off = lay.gu_scale_offset;
+    a.kblocks = d->H / 128;
+    if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H, kBoxN)) != MOE_OK) return st;
+    if ((st = encode_act_map(&a.act_map64, x_perm, rows, d->H, 64)) != MOE_OK) return st;
     a.K = d->H;
     a.M = d->I;
     a.up_row = d->I;
     a.out = static_cast<__nv_bfloat16*>(h);
     a.ld_out = d->I;
-    if ((st = launch_bn<kGated>(bn, a, (int)rows, G, stream)) != MOE_OK) return st;
+    if ((st = launch_w<kGated>(w8, bn, a, (int)rows, G, stream)) != MOE_OK) return st;
 
     // GEMM2: y = h W_down^T
     for (int q = 0; q < 2; ++q)
         if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.down_offset,
-                                                    count[q], stride[q], d->I, d->H)) != MOE_OK)
+                                                    count[q], stride[q], d->I, d->H, w8)) != MOE_OK)
             return st;
     if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.down_offset, 1,
-                                                 lay.bytes, d->I, d->H)) != MOE_OK)
+                                                 lay.bytes, d->I, d->H, w8)) != MOE_OK)
         return st;
-    if ((st = encode_act_map(&a.act_map, h, rows, d->I)) != MOE_OK) return st;
+    a.scale_off = lay.down_scale_offset;
+    a.kblocks = d->I / 128;
+    if ((st = encode_act_map(&a.act_map, h, rows, d->I, kBoxN)) != MOE_OK) return st;
+    if ((st = encode_act_map(&a.act_map64, h, rows, d->I, 64)) != MOE_OK) return st;
     a.K = d->I;
     a.M = d->H;
     a.up_row = 0;
     a.out = static_cast<__nv_bfloat16*>(y_perm);
     a.ld_out = d->H;
-    if (d->H % (2 * kBM) == 0) return launch_bn<kPair>(bn, a, (int)rows, G, stream);
-    return launch_bn<kSingle>(bn, a, (int)rows, G, stream);
+    if (d->H % (2 * kBM) == 0) return launch_w<kPair>(w8, bn, a, (int)rows, G, stream);
+    return launch_w<kSingle>(w8, bn, a, (int)rows, G, stream);
 }
 
 }  // extern "C"

@@ -55,7 +55,6 @@ __global__ void __launch_bounds__(kThreads) k_hist(const int32_t* __restrict__ i
 __global__ void __launch_bounds__(1024) k_scan(const int32_t* __restrict__ blk_counts, int nb,
                                                int E, int32_t* __restrict__ blk_base,
                                                int32_t* __restrict__ offsets) {
-    __shared__ int total[MOE_MAX_EXPERTS];
     __shared__ int warp_sums[32];
     const int e = threadIdx.x;
     int run = 0;
@@ -88,7 +87,6 @@ __global__ void __launch_bounds__(1024) k_scan(const int32_t* __restrict__ blk_c
     __syncthreads();
     const int excl = warp_sums[warp] + incl - v;
     if (e < E) {
-        total[e] = excl;
         offsets[e] = excl;
         if (e == E - 1) offsets[E] = excl + v;
         for (int b = 0; b < nb; ++b) blk_base[(int64_t)b * E + e] += excl;
@@ -139,28 +137,12 @@ __global__ void __launch_bounds__(kThreads) k_scatter(const int32_t* __restrict_
     }
 }
 
-template <typename T>
-__device__ __forceinline__ void load8(const T* row, int c, float (&v)[8]);
-
-template <>
-__device__ __forceinline__ void load8<float>(const float* row, int c, float (&v)[8]) {
+// Eight consecutive fp32 values as two 16-byte loads.
+__device__ __forceinline__ void load8(const float* row, int c, float (&v)[8]) {
     const float4 a = *reinterpret_cast<const float4*>(row + c);
     const float4 b = *reinterpret_cast<const float4*>(row + c + 4);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* row, int c,
-                                                     float (&v)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(row + c);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h[i]);
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
-    }
 }
 
 // One warp per output row; 8 columns (one 16-byte bf16 vector) per lane step.

@@ -97,6 +97,114 @@ __global__ void __launch_bounds__(256) k_logits(const XT* __restrict__ x,
     }
 }
 
+// Large batches: a 128-token x 128-expert block tile, 8 x 8 (token, expert)
+// pairs per thread, 16 h per shared-memory stage with the next stage's
+// global loads held in registers while the current one is consumed.  The
+// arithmetic order is the same as k_logits: per 256-wide chunk a fused
+// multiply-add chain in ascending h, chunk sums added in ascending order.
+constexpr int kBigT = 128, kBigE = 128, kBigK = 16;
+
+constexpr int kBigLd = kBigE + 4;  // row stride of the running sums in shared memory
+constexpr size_t kBigDynSmem = (size_t)kBigT * kBigLd * sizeof(float);
+
+template <typename XT>
+__global__ void __launch_bounds__(256, 1) k_logits_big(const XT* __restrict__ x,
+                                                       const float* __restrict__ wg, int T, int H,
+                                                       int E, float* __restrict__ out) {
+    __shared__ __align__(16) float xs[2][kBigK][kBigT + 4];
+    __shared__ __align__(16) float ws[2][kBigK][kBigE + 4];
+    extern __shared__ float ls[];  // [kBigT][kBigLd]: sum of the finished chunks, per pair
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int e0 = blockIdx.x * kBigE, t0 = blockIdx.y * kBigT;
+    // loader mapping: x  -> token lt = tid / 2, h offset (tid % 2) * 8   (8 values)
+    //                 w  -> expert le = tid / 2, h offset (tid % 2) * 8   (8 values)
+    const int lt = tid >> 1, lh = (tid & 1) * 8;
+    const bool xin = t0 + lt < T, win = e0 + lt < E;
+    const XT* xrow = x + (int64_t)(xin ? t0 + lt : 0) * H + lh;
+    const float* wrow = wg + (int64_t)(win ? e0 + lt : 0) * H + lh;
+    float rx[8], rw[8];
+    auto load = [&](int h0) {
+        if constexpr (sizeof(XT) == 2) {
+            const uint4 u = xin ? *reinterpret_cast<const uint4*>(xrow + h0) : make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b2[i]);
+                rx[2 * i] = f.x;
+                rx[2 * i + 1] = f.y;
+            }
+        } else {
+            const float4 a = xin ? *reinterpret_cast<const float4*>(xrow + h0) : make_float4(0, 0, 0, 0);
+            const float4 b = xin ? *reinterpret_cast<const float4*>(xrow + h0 + 4) : make_float4(0, 0, 0, 0);
+            rx[0] = a.x; rx[1] = a.y; rx[2] = a.z; rx[3] = a.w;
+            rx[4] = b.x; rx[5] = b.y; rx[6] = b.z; rx[7] = b.w;
+        }
+        const float4 a = win ? *reinterpret_cast<const float4*>(wrow + h0) : make_float4(0, 0, 0, 0);
+        const float4 b = win ? *reinterpret_cast<const float4*>(wrow + h0 + 4) : make_float4(0, 0, 0, 0);
+        rw[0] = a.x; rw[1] = a.y; rw[2] = a.z; rw[3] = a.w;
+        rw[4] = b.x; rw[5] = b.y; rw[6] = b.z; rw[7] = b.w;
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            xs[buf][lh + i][lt] = rx[i];
+            ws[buf][lh + i][lt] = rw[i];
+        }
+    };
+    auto row_of = [&](int i) { return i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4; };
+    auto col_of = [&](int j) { return j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4; };
+    float p[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) p[i][j] = 0.0f;
+    const int nk = H / kBigK;
+    load(0);
+    store(0);
+    __syncthreads();
+    for (int kt = 0; kt < nk; ++kt) {
+        const int buf = kt & 1;
+        if (kt + 1 < nk) load((kt + 1) * kBigK);
+#pragma unroll
+        for (int kk = 0; kk < kBigK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&ws[buf][kk][64 + tx * 4]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) p[i][j] = __fmaf_rn(a[i], b[j], p[i][j]);
+        }
+        const int h_next = (kt + 1) * kBigK;
+        if (h_next % kChunk == 0 || h_next >= H) {  // a 256-wide chunk ends here
+            const bool first = (h_next - 1) / kChunk == 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float* l = &ls[row_of(i) * kBigLd + col_of(j)];
+                    *l = first ? p[i][j] : __fadd_rn(*l, p[i][j]);
+                    p[i][j] = 0.0f;
+                }
+        }
+        if (kt + 1 < nk) store(buf ^ 1);
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + row_of(i);
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = e0 + col_of(j);
+            if (e < E) out[(int64_t)t * E + e] = ls[row_of(i) * kBigLd + col_of(j)];
+        }
+    }
+}
+
 // e^y in fp64 for |y| <= 700, every step one IEEE operation: Cody-Waite
 // reduction with ln 2 = LN2_HI + LN2_LO (LN2_HI has 21 trailing zero bits),
 // Taylor polynomial to degree 13 by Horner, exact scaling by 2^n.
@@ -158,16 +266,26 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ logits
     const float kNegInf = -__int_as_float(0x7f800000);
     float lg[V], key[V], sc[V];
     bool cand[V];
+    // l = P_0 + P_1 + ... in chunk order; the loads of one chunk for all of
+    // this lane's experts are independent and issued together
 #pragma unroll
     for (int v = 0; v < V; ++v) {
         const int e = lane + 32 * v;
-        lg[v] = kNegInf;
-        if (e < E) {
-            float acc = logits[(int64_t)t * E + e];
-            for (int c = 1; c < nsplit; ++c)
-                acc = __fadd_rn(acc, logits[((int64_t)c * T + t) * E + e]);
-            lg[v] = acc;
-        }
+        lg[v] = (e < E) ? logits[(int64_t)t * E + e] : kNegInf;
+    }
+#pragma unroll 2
+    for (int c = 1; c < nsplit; ++c) {
+        const float* part = logits + ((int64_t)c * T + t) * E;
+        float pc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) pc[v] = (lane + 32 * v < E) ? part[lane + 32 * v] : 0.0f;
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+            if (lane + 32 * v < E) lg[v] = __fadd_rn(lg[v], pc[v]);
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        const int e = lane + 32 * v;
         if (score == MOE_SCORE_SIGMOID) {
             sc[v] = (e < E) ? sigmoid_f32(lg[v]) : 0.0f;
             key[v] = (e < E) ? (bias ? __fadd_rn(sc[v], bias[e]) : sc[v]) : kNegInf;
@@ -269,15 +387,18 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ logits
 }
 
 struct RoutePlan {
-    int tm;      // 2 or 4 (TM == TN)
+    int tm;      // 2 or 4 (k_logits, TM == TN) or 8 (k_logits_big)
     int nsplit;  // 1, or the number of 256-wide chunks
 };
 
+// Small batches split the h chunks over the grid (partial sums added in
+// order by k_select); large ones use the 128 x 128 tile when it fills the GPU.
 RoutePlan plan(const moe_route_cfg* c) {
     RoutePlan p;
     const int64_t tiles32 = (int64_t)((c->T + 31) / 32) * ((c->E + 31) / 32);
+    const int64_t tiles128 = (int64_t)((c->T + kBigT - 1) / kBigT) * ((c->E + kBigE - 1) / kBigE);
     const bool small = tiles32 < 512;
-    p.tm = small ? 2 : 4;
+    p.tm = small ? 2 : (tiles128 >= 120 ? 8 : 4);
     p.nsplit = small ? (c->H + kChunk - 1) / kChunk : 1;
     return p;
 }
@@ -310,10 +431,16 @@ void launch_logits(const moe_route_cfg* c, const RoutePlan& p, const XT* x, cons
                    float* out, cudaStream_t s) {
     const int B = 16 * p.tm;
     dim3 grid((c->E + B - 1) / B, (c->T + B - 1) / B, p.nsplit);
-    if (p.tm == 2)
+    if (p.tm == 8) {
+        dim3 g((c->E + kBigE - 1) / kBigE, (c->T + kBigT - 1) / kBigT);
+        cudaFuncSetAttribute(k_logits_big<XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kBigDynSmem);
+        k_logits_big<XT><<<g, 256, kBigDynSmem, s>>>(x, wg, c->T, c->H, c->E, out);
+    } else if (p.tm == 2) {
         k_logits<XT, 2, 2><<<grid, 256, 0, s>>>(x, wg, c->T, c->H, c->E, p.nsplit > 1, out);
-    else
+    } else {
         k_logits<XT, 4, 4><<<grid, 256, 0, s>>>(x, wg, c->T, c->H, c->E, p.nsplit > 1, out);
+    }
 }
 
 }  // namespace

@@ -19,6 +19,10 @@ MID_SOFTMAX = config(1).with_(cfg_id=12, name="mid_softmax_f32_T257_H384_I256_E1
                               I=256, E=16, k=3, local_count=6)
 SPARSE_DECODE = config(2).with_(cfg_id=13, name="sparse_decode_T5_H256_I128_E64", T=5, H=256,
                                 I=128, E=64, k=8, n_group=8, topk_group=4, local_count=16)
+MID_FP8 = config(5).with_(cfg_id=24, name="mid_fp8_T300_H512_I256_E32", T=300, H=512, I=256,
+                          E=32, k=4, n_group=4, topk_group=2, local_count=8, layers=1)
+DECODE_FP8 = config(5).with_(cfg_id=25, name="decode_fp8_T7_H256_I128_E64", T=7, H=256, I=128,
+                             E=64, k=8, n_group=8, topk_group=4, local_count=16, layers=1)
 ONE_TOKEN = config(2).with_(cfg_id=14, name="one_token_H256_I256_E16", T=1, H=256, I=256, E=16,
                             k=2, n_group=4, topk_group=2, local_count=4)
 

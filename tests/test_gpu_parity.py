@@ -15,8 +15,8 @@ from moe_inputs import config, device as mdev, gen
 from oracle import workload as ow
 from split_weight_b200 import _lib as L
 
-from gpu_util import (MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16, SPARSE_DECODE,
-                      assert_close_rel, run_layer, sync_check, to_np)
+from gpu_util import (DECODE_FP8, MID_FP8, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16,
+                      RTOL_FP8, SPARSE_DECODE, assert_close_rel, run_layer, sync_check, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -56,14 +56,18 @@ def _check_permutation(dl, idx_ref):
         np.testing.assert_array_equal(xp[c.A:], xb)
 
 
-@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def _rtol(cfg):
+    return RTOL_FP8 if cfg.w_dtype == "e4m3" else RTOL_BF16
+
+
+@pytest.mark.parametrize("cfg", SMALL + [MID_FP8, DECODE_FP8], ids=lambda c: c.name)
 def test_small_layer_full_parity(cfg):
     dl = mdev.build_layer(cfg)
     run_layer(dl)
     y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
     _check_routing(dl, idx_ref, w_ref)
     _check_permutation(dl, idx_ref)
-    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, RTOL_BF16, f"{cfg.name} y")
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
 
 
 def test_generator_gpu_matches_host(cuda_device):
@@ -151,7 +155,7 @@ def _full_size_check(cfg, layer: int, n_sample: int = 12):
     toks = np.sort(rng.choice(cfg.T, size=min(n_sample, cfg.T), replace=False))
     y_ref = ow.layer_tokens(cfg, layer, toks, idx_ref, w_ref, dl.pool, dl.slot, dl.inputs)
     y = to_np(dl.layer.y[torch.from_numpy(toks).cuda()])
-    return assert_close_rel(y, y_ref, RTOL_BF16, f"{cfg.name} layer {layer} sampled y")
+    return assert_close_rel(y, y_ref, _rtol(cfg), f"{cfg.name} layer {layer} sampled y")
 
 
 def test_r1_decode_full_size():
@@ -165,3 +169,81 @@ def test_r1_prefill_8k_full_size():
 @pytest.mark.parametrize("layer", [0, 1])
 def test_r1_prefill_imbalanced_full_size(layer):
     _full_size_check(config(4), layer, n_sample=6)
+
+
+@pytest.mark.parametrize("layer", [0, 3])
+def test_r1_fp8_pipeline_full_size(layer):
+    _full_size_check(config(5), layer, n_sample=6)
+
+
+def test_e4m3_gather_quantises_each_128_block(cuda_device):
+    """moe_permute with an e4m3 destination: the permutation is exact and each
+    row's 128-column blocks decode to within e4m3 rounding of x."""
+    cfg = MID_SIGMOID
+    li = gen.layer_inputs(cfg)
+    idx_ref, _, _ = ow.route(cfg, 0, li)
+    T, k, E, H = cfg.T, cfg.k, cfg.E, cfg.H
+    rows = T * k + T
+    dev = cuda_device
+    idx = torch.from_numpy(idx_ref).to(dev)
+    x = mdev.x_tensor(li, dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    src = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T, k, dtype=torch.int32, device=dev)
+    xq = torch.empty(rows, H, dtype=torch.uint8, device=dev)
+    sc = torch.empty(rows, H // 128, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=dev)
+    L.check(L.moe_permute(T, k, E, H, idx.data_ptr(), x.data_ptr(), L.MOE_BF16, L.MOE_E4M3, 1,
+                          off.data_ptr(), src.data_ptr(), inv.data_ptr(), xq.data_ptr(),
+                          sc.data_ptr(), ws.data_ptr(), ws.numel(),
+                          torch.cuda.current_stream().cuda_stream))
+    sync_check()
+    o_ref, s_ref, _ = oracle.permute(idx_ref, E)
+    np.testing.assert_array_equal(src.cpu().numpy(), s_ref)
+    xs = np.concatenate([li.x[s_ref], li.x]).astype(np.float64)
+    dec = gen.e4m3_bits_to_f64(xq.cpu().numpy()) * np.repeat(sc.cpu().numpy(), 128, axis=1)
+    blk = np.abs(xs).reshape(rows, H // 128, 128).max(axis=2)
+    np.testing.assert_allclose(sc.cpu().numpy(), blk / 448, rtol=1e-6)
+    # e4m3 has 3 mantissa bits: |err| <= 2^-4 |v| for normal codes, plus the
+    # subnormal step 2^-10 * s
+    bound = np.abs(xs) * 2.0 ** -4 + np.repeat(sc.cpu().numpy(), 128, axis=1) * 2.0 ** -10
+    assert (np.abs(dec - xs) <= bound * (1 + 1e-6)).all()
+
+
+# ----------------------------------------------------------------- routing only
+BIG_ROUTE_BF16 = config(2).with_(cfg_id=18, name="route_T7700_H512_E256", T=7700, H=512, I=128)
+BIG_ROUTE_F32 = config(1).with_(cfg_id=19, name="route_f32_T20000_H256_E8", T=20000)
+MED_ROUTE = config(2).with_(cfg_id=22, name="route_T3001_H512_E256", T=3001, H=512, I=128)
+SPLIT_ROUTE = config(2).with_(cfg_id=20, name="route_T40_H7168_E256", T=40, I=128)
+
+
+@pytest.mark.parametrize("cfg", [BIG_ROUTE_BF16, BIG_ROUTE_F32, MED_ROUTE, SPLIT_ROUTE],
+                         ids=lambda c: c.name)
+def test_routing_bit_exact_all_router_kernels(cfg, cuda_device):
+    """The three logits kernels (chunk-split for small batches, 64x64 and
+    128x128 tiles for large ones, ragged token counts) give the oracle's
+    bits; so do the selection and the permutation that follow."""
+    from moe_inputs.gen import layer_inputs
+    from split_weight_b200 import MoELayer, SplitWeights
+    li = layer_inputs(cfg)
+    shape = mdev.layer_shape(cfg)
+    w = SplitWeights.allocate(cfg.H, cfg.I, cfg.w_dtype, *mdev.default_placement(cfg),
+                              cfg.has_shared, cuda_device)
+    bias = torch.from_numpy(li.bias).to(cuda_device) if li.bias is not None else None
+    ml = MoELayer(shape, torch.from_numpy(li.wg).to(cuda_device), bias, w, cuda_device)
+    x = mdev.x_tensor(li, cuda_device)
+    h = torch.cuda.current_stream().cuda_stream
+    ml.route(x, h)
+    ml.permute(x, h)
+    sync_check()
+    idx_ref, w_ref, _ = ow.route(cfg, 0, li)
+    np.testing.assert_array_equal(ml.topk_idx[:cfg.T].cpu().numpy(), idx_ref)
+    got_w = ml.topk_w[:cfg.T].cpu().numpy()
+    if cfg.score == "sigmoid":
+        np.testing.assert_array_equal(got_w, w_ref.astype(np.float32))
+    else:
+        np.testing.assert_allclose(got_w, w_ref, rtol=2e-6, atol=1e-7)
+    off, src, inv = oracle.permute(idx_ref, cfg.E)
+    np.testing.assert_array_equal(ml.offsets.cpu().numpy(), off)
+    np.testing.assert_array_equal(ml.perm_src[:cfg.A].cpu().numpy(), src)
+    np.testing.assert_array_equal(ml.inv_pos[:cfg.T].cpu().numpy(), inv)
