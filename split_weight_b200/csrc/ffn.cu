@@ -65,7 +65,7 @@ struct alignas(64) FfnArgs {
 enum { kSingle = 0, kGated = 1, kPair = 2 };
 
 constexpr uint32_t kA8Bytes = kBM * kBK;       // one e4m3 weight tile as loaded, 8 KB
-constexpr int kConvThreads = 128;              // e4m3 -> bf16 converter warps (4)
+constexpr int kConvThreads = 256;              // e4m3 -> bf16 converter warps (8)
 
 // Per stage: the bf16 weight tile(s) the MMA reads (128-byte swizzled), the
 // token tile, and for e4m3 weights the staging tile(s) TMA writes.
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         // row is 128 bytes in the 128-byte swizzle: 16-byte chunk j of row r
         // sits at position j ^ (r % 8).  One 128x128 block scale covers the
         // whole stage (64 columns of K, 128 rows).
-        const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. 127
+        const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. kConvThreads-1
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 for (int a = 0; a < C::kNA; ++a) {
                     const float sc = a == 0 ? s0 : s1;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < (kBM * kBK / 16) / kConvThreads; ++i) {
                         const int id = ct + kConvThreads * i, r = id >> 2, c = id & 3;
                         uint4 in, lo, hi;
                         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"

@@ -23,6 +23,9 @@ MID_FP8 = config(5).with_(cfg_id=24, name="mid_fp8_T300_H512_I256_E32", T=300, H
                           E=32, k=4, n_group=4, topk_group=2, local_count=8, layers=1)
 DECODE_FP8 = config(5).with_(cfg_id=25, name="decode_fp8_T7_H256_I128_E64", T=7, H=256, I=128,
                              E=64, k=8, n_group=8, topk_group=4, local_count=16, layers=1)
+# the largest shapes the ABI takes: 1024 experts, k = 32, 32 groups (one per lane)
+MAX_EXPERTS = config(2).with_(cfg_id=26, name="max_E1024_k32_G32_T64", T=64, H=256, I=128,
+                              E=1024, k=32, n_group=32, topk_group=4, local_count=256)
 ONE_TOKEN = config(2).with_(cfg_id=14, name="one_token_H256_I256_E16", T=1, H=256, I=256, E=16,
                             k=2, n_group=4, topk_group=2, local_count=4)
 

@@ -15,7 +15,7 @@ from moe_inputs import config, device as mdev, gen
 from oracle import workload as ow
 from split_weight_b200 import _lib as L
 
-from gpu_util import (DECODE_FP8, MID_FP8, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16,
+from gpu_util import (DECODE_FP8, MAX_EXPERTS, MID_FP8, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16,
                       RTOL_FP8, SPARSE_DECODE, assert_close_rel, run_layer, sync_check, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -60,7 +60,7 @@ def _rtol(cfg):
     return RTOL_FP8 if cfg.w_dtype == "e4m3" else RTOL_BF16
 
 
-@pytest.mark.parametrize("cfg", SMALL + [MID_FP8, DECODE_FP8], ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", SMALL + [MID_FP8, DECODE_FP8, MAX_EXPERTS], ids=lambda c: c.name)
 def test_small_layer_full_parity(cfg):
     dl = mdev.build_layer(cfg)
     run_layer(dl)
