@@ -135,7 +135,9 @@ MOE_API moe_status moe_route(const moe_route_cfg *cfg, const void *x, moe_dtype 
  *   the always-on shared expert).
  * perm_dtype MOE_BF16: x_perm [rows, H] bf16 (fp32 x is rounded to nearest
  * even).  perm_dtype MOE_E4M3: x_perm [rows, H] e4m3 plus x_perm_scales
- * [rows, H/128] fp32, per 128 columns s = amax/448, code = e4m3(v/s).
+ * [H/128, rows] fp32 (one row of scales per 128-column block, so a block's
+ * scales for consecutive rows are contiguous): per row and 128 columns
+ * s = amax/448, code = e4m3(v/s).
  * topk_idx entries must lie in [0, E) (checked on the device: an entry
  * outside sets the device error word, MOE_ERR_DEVICE_CHECK, and is skipped).
  * Limits: H % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.

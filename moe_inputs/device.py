@@ -38,13 +38,14 @@ def random_placement(cfg: MoEConfig, seed: int, n_local: int | None = None):
     return pool, slot
 
 
-def layer_shape(cfg: MoEConfig):
+def layer_shape(cfg: MoEConfig, act_dtype: str | None = None):
     from split_weight_b200 import LayerShape
     return LayerShape(T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k, score=cfg.score,
                       n_group=cfg.n_group, topk_group=cfg.topk_group,
                       routed_scale=cfg.routed_scale, renormalize=cfg.renormalize,
                       has_shared=cfg.has_shared, x_dtype=cfg.x_dtype, w_dtype=cfg.w_dtype,
-                      y_dtype="f32" if cfg.x_dtype == "f32" else "bf16")
+                      y_dtype="f32" if cfg.x_dtype == "f32" else "bf16",
+                      act_dtype=act_dtype or ("e4m3" if cfg.w_dtype == "e4m3" else "bf16"))
 
 
 def x_tensor(li: gen.LayerInputs, device) -> torch.Tensor:
@@ -75,7 +76,8 @@ class DeviceLayer:
     slot: np.ndarray
 
 
-def build_layer(cfg, layer: int = 0, device="cuda", placement=None) -> DeviceLayer:
+def build_layer(cfg, layer: int = 0, device="cuda", placement=None,
+                act_dtype: str | None = None) -> DeviceLayer:
     from split_weight_b200 import MoELayer, SplitWeights
     cfg = config(cfg)
     li = gen.layer_inputs(cfg, layer)
@@ -84,7 +86,7 @@ def build_layer(cfg, layer: int = 0, device="cuda", placement=None) -> DeviceLay
     fill_weights(cfg, layer, w)
     wg = torch.from_numpy(li.wg).to(device)
     bias = torch.from_numpy(li.bias).to(device) if li.bias is not None else None
-    ml = MoELayer(layer_shape(cfg), wg, bias, w, device)
+    ml = MoELayer(layer_shape(cfg, act_dtype), wg, bias, w, device)
     return DeviceLayer(cfg, layer, li, x_tensor(li, device), ml, pool, slot)
 
 

@@ -60,6 +60,13 @@ struct alignas(64) FfnArgs {
     int64_t w_stride[3];
     int64_t scale_off;
     int32_t kblocks;
+    // e4m3 activations (tensor-core fp8 path): activation scales [K/128][act_scale_ld]
+    // (row = permuted row), and for the gate/up kernel the e4m3 output h with its
+    // scales [M/128][act_scale_ld]
+    const float* act_scale;
+    int32_t act_scale_ld;
+    uint8_t* out8;
+    float* out_scale;
 };
 
 enum { kSingle = 0, kGated = 1, kPair = 2 };
@@ -89,6 +96,34 @@ struct Cfg {
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                   "TMEM allocation must be a power of two in [32, 512]");
     static_assert(kStages >= 2, "pipeline needs two stages");
+};
+
+// e4m3 weights and e4m3 activations on the tensor cores (kind::f8f6f4).
+// A stage is one 128 x 128 scale block of K; its MMAs go into a fresh TMEM
+// partial sum, which the epilogue warps fold into fp32 registers with the
+// block's scales (weight block scale x per-token activation scale).
+template <int BN, int MODE>
+struct CfgF8 {
+    static constexpr int kNA = 2;                                   // GATED or PAIR
+    static constexpr int kBK8 = 128;                                // K (bytes) per stage
+    static constexpr uint32_t kATile = kBM * kBK8;                  // 16 KB
+    static constexpr uint32_t kAStage = kATile * kNA;
+    static constexpr uint32_t kBStage = BN * kBK8;
+    static constexpr uint32_t kStageBytes = kAStage + kBStage;
+    static constexpr int kStages = (kSmemBudget / kStageBytes) > 8 ? 8 : (kSmemBudget / kStageBytes);
+    static constexpr uint32_t kPartCols = kNA * BN;                 // one partial-sum set
+    static constexpr int kPBufs = (512 / kPartCols) >= 8 ? 8 : (512 / kPartCols);
+    static constexpr uint32_t kTmemCols = kPBufs * kPartCols;
+    static constexpr int kEpiWarps = 8;                             // 2 per TMEM lane quarter
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    static constexpr int kRowsPerTile = MODE == kPair ? 2 * kBM : kBM;
+    static constexpr int kCols = BN / 2;                            // columns per epilogue warp
+    // per-warp combined scales [8][2][kCols] + amax exchange [2 halves][2 tiles][4][kCols]
+    static constexpr size_t kScratch = (size_t)kEpiWarps * 2 * kCols * 4 + 2 * 2 * 4 * kCols * 4;
+    static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024 + kScratch;
+    static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                  "TMEM allocation must be a power of two in [32, 512]");
+    static_assert(kStages >= 2 && BN <= 128 && BN % 16 == 0, "fp8 tile shape");
 };
 
 struct Tile {
@@ -139,6 +174,43 @@ __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
     t.map = tb.ps[g] >> 24;
     t.slot = tb.ps[g] & 0xFFFFFF;
     return t;
+}
+
+// One warp: per-group first row, rows, tile count and (pool, slot), and the
+// exclusive scan of tiles over the groups (routed experts, then the shared one).
+template <int BN>
+__device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G, int MT, int lane) {
+    const int per = (G + 31) / 32, g0 = lane * per, g1 = min(G, g0 + per);
+    int sum = 0;
+    for (int g = g0; g < g1; ++g) {
+        int n, r0, ps;
+        if (g < p.E) {
+            r0 = p.offsets[g];
+            n = p.offsets[g + 1] - r0;
+            const uint32_t v = static_cast<uint32_t>(p.pool_slot[g]);
+            ps = (int)(((v >> 31) << 24) | (v & 0xFFFFFFu));
+        } else {
+            r0 = p.A;
+            n = p.T;
+            ps = 2 << 24;
+        }
+        tb.row0[g] = r0;
+        tb.n[g] = n;
+        tb.ps[g] = ps;
+        sum += token_tiles<BN>(n) * MT;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+    for (int g = g0; g < g1; ++g) {
+        tb.tile_start[g] = run;
+        run += token_tiles<BN>(tb.n[g]) * MT;
+    }
+    if (lane == 31) tb.tile_start[G] = incl;
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
@@ -202,40 +274,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 2) {
-        // per-group rows, tiles and (pool, slot); exclusive scan of tiles
-        const int per = (G + 31) / 32, g0 = lane * per, g1 = min(G, g0 + per);
-        int sum = 0;
-        for (int g = g0; g < g1; ++g) {
-            int n, r0, ps;
-            if (g < p.E) {
-                r0 = p.offsets[g];
-                n = p.offsets[g + 1] - r0;
-                const uint32_t v = static_cast<uint32_t>(p.pool_slot[g]);
-                ps = (int)(((v >> 31) << 24) | (v & 0xFFFFFFu));
-            } else {
-                r0 = p.A;
-                n = p.T;
-                ps = 2 << 24;
-            }
-            tb.row0[g] = r0;
-            tb.n[g] = n;
-            tb.ps[g] = ps;
-            sum += token_tiles<BN>(n) * MT;
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - sum;
-        for (int g = g0; g < g1; ++g) {
-            tb.tile_start[g] = run;
-            run += token_tiles<BN>(tb.n[g]) * MT;
-        }
-        if (lane == 31) tb.tile_start[G] = incl;
-    }
+    if (warp == 2) build_tables<BN>(p, tb, G, MT, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -442,6 +481,289 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------- fp8 tensor-core kernel
+// warp 0 TMA producer, warp 1 MMA issuer, warps 2..9 epilogue.  Every stage
+// (one 128-wide block of K) is multiplied into a fresh TMEM partial sum; the
+// epilogue warps fold it into fp32 registers as acc += P * s_w * s_x[token],
+// where s_w is the 128 x 128 weight block scale and s_x the activation
+// scale of the token for that block of K.  GATED then quantises
+// h = silu(gate) * up to e4m3 per (token, 128 features) for the down GEMM;
+// PAIR writes bf16.
+template <int BN, int MODE>
+__global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
+    k_grouped_ffn_f8(const __grid_constant__ FfnArgs p) {
+    using C = CfgF8<BN, MODE>;
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
+    __shared__ __align__(8) uint64_t part_full[C::kPBufs], part_empty[C::kPBufs];
+    __shared__ __align__(8) uint64_t half_bar[2];   // the 4 epilogue warps of one column half
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ Tables tb;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t base_addr = smem_u32(dyn_smem);
+    const uint32_t stages = (base_addr + 1023u) & ~1023u;
+    float* scratch = reinterpret_cast<float*>(dyn_smem + (stages - base_addr) +
+                                              (size_t)C::kStages * C::kStageBytes);
+    const int G = p.E + (p.has_shared ? 1 : 0);
+    const int MT = p.M / C::kRowsPerTile;
+    const int KB = p.K / C::kBK8;
+    volatile int* abort_flag = &abort_sh;
+
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int b = 0; b < C::kPBufs; ++b) {
+            mbar_init(smem_u32(&part_full[b]), 1);
+            mbar_init(smem_u32(&part_empty[b]), C::kEpiWarps);
+        }
+        mbar_init(smem_u32(&half_bar[0]), 4);
+        mbar_init(smem_u32(&half_bar[1]), 4);
+        fence_mbar_init();
+        tma_prefetch_map(&p.act_map);
+        tma_prefetch_map(&p.act_map64);
+        for (int m = 0; m < 3; ++m) tma_prefetch_map(&p.w_map[m]);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 2) build_tables<BN>(p, tb, G, MT, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+    const int total = tb.tile_start[G];
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+                const CUtensorMap* wm = &p.w_map[t.map];
+                const uint32_t tx = C::kAStage + (uint32_t)t.n_mma * C::kBK8;
+                const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    mbar_arrive_expect_tx(fb, tx);
+                    tma_load_3d(sa, wm, fb, kb * C::kBK8, t.m0, t.slot);
+                    tma_load_3d(sa + C::kATile, wm, fb, kb * C::kBK8, row_a1, t.slot);
+                    const uint32_t sb = sa + C::kAStage;
+                    int r = 0;
+                    for (; r + 64 <= t.n_mma; r += 64)
+                        tma_load_2d(sb + r * C::kBK8, &p.act_map64, fb, kb * C::kBK8, t.row0 + r);
+                    for (; r < t.n_mma; r += kBoxN)
+                        tma_load_2d(sb + r * C::kBK8, &p.act_map, fb, kb * C::kBK8, t.row0 + r);
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, pb = 0;
+            uint32_t phase = 0, use[C::kPBufs];
+#pragma unroll
+            for (int b = 0; b < C::kPBufs; ++b) use[b] = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+                const uint32_t idesc = idesc_e4m3_f32(kBM, t.n_mma);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(smem_u32(&part_empty[pb]), (use[pb] & 1u) ^ 1u, abort_flag, p.err) ||
+                        !mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    const uint32_t sb = sa + C::kAStage;
+                    const uint32_t d0 = tmem_base + pb * C::kPartCols;
+#pragma unroll
+                    for (int kk = 0; kk < C::kBK8 / 32; ++kk) {
+                        const uint64_t bd = sw128_desc(sb + kk * 32);
+                        mma_e4m3_ss(d0, sw128_desc(sa + kk * 32), bd, idesc, kk != 0);
+                        mma_e4m3_ss(d0 + BN, sw128_desc(sa + C::kATile + kk * 32), bd, idesc, kk != 0);
+                    }
+                    mma_commit(smem_u32(&empty_bar[stage]));
+                    mma_commit(smem_u32(&part_full[pb]));
+                    ++use[pb];
+                    if (++pb == C::kPBufs) pb = 0;
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..9)
+        constexpr int kC = C::kCols;
+        const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int part = (warp - 2) >> 2;    // which half of the token columns
+        const int e = warp - 2;
+        const int c_begin = part * kC;
+        float* cg = scratch + e * 2 * kC;    // this warp's combined scales, gate / row block 0
+        float* cu = cg + kC;                 //                              up / row block 1
+        float* red_half = scratch + C::kEpiWarps * 2 * kC + part * 2 * 4 * kC;  // [2][4][kC]
+        uint32_t tiles_done = 0;
+        int pb = 0;
+        uint32_t use[C::kPBufs];
+#pragma unroll
+        for (int b = 0; b < C::kPBufs; ++b) use[b] = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+            const uint8_t* sbase = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map] + p.scale_off;
+            const float* sw0p = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
+            const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
+            const float* sw1p = reinterpret_cast<const float*>(sbase) + (int64_t)rb1 * p.kblocks;
+            // this lane's token columns of the activation scales: c_begin + lane + 32 i
+            constexpr int kSx = (kC + 31) / 32;
+            auto load_sx = [&](int kb, float (&sx)[kSx]) {
+#pragma unroll
+                for (int i = 0; i < kSx; ++i) {
+                    const int col = c_begin + lane + 32 * i;
+                    const int r = t.row0 + col;
+                    sx[i] = (lane + 32 * i < kC && col < t.n_rows)
+                                ? __ldg(p.act_scale + (int64_t)kb * p.act_scale_ld + r) : 0.0f;
+                }
+            };
+            float acc0[kC], acc1[kC];
+#pragma unroll
+            for (int j = 0; j < kC; ++j) acc0[j] = acc1[j] = 0.0f;
+            float sx[kSx], sxn[kSx];
+            load_sx(0, sx);
+            float sw0 = __ldg(sw0p), sw1 = __ldg(sw1p);
+            for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+                for (int i = 0; i < kSx; ++i) {
+                    if (lane + 32 * i < kC) {
+                        cg[lane + 32 * i] = sx[i] * sw0;
+                        cu[lane + 32 * i] = sx[i] * sw1;
+                    }
+                }
+                __syncwarp();
+                float sw0n = 0.0f, sw1n = 0.0f;
+                if (kb + 1 < KB) {   // next block's scales travel while this one is folded in
+                    load_sx(kb + 1, sxn);
+                    sw0n = __ldg(sw0p + kb + 1);
+                    sw1n = __ldg(sw1p + kb + 1);
+                }
+                ok = mbar_wait(smem_u32(&part_full[pb]), use[pb] & 1u, abort_flag, p.err);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tp = tmem_base + ((uint32_t)(32 * q) << 16) + pb * C::kPartCols + c_begin;
+#pragma unroll
+                for (int c0 = 0; c0 < kC; c0 += 8) {
+                    float a[8], b[8];
+                    tmem_ld_8(tp + c0, a);
+                    tmem_ld_8(tp + BN + c0, b);
+                    tmem_ld_wait();
+                    const float4 g0 = *reinterpret_cast<const float4*>(cg + c0);
+                    const float4 g1 = *reinterpret_cast<const float4*>(cg + c0 + 4);
+                    const float4 u0 = *reinterpret_cast<const float4*>(cu + c0);
+                    const float4 u1 = *reinterpret_cast<const float4*>(cu + c0 + 4);
+                    const float gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const float us[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        acc0[c0 + i] = fmaf(a[i], gs[i], acc0[c0 + i]);
+                        acc1[c0 + i] = fmaf(b[i], us[i], acc1[c0 + i]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&part_empty[pb]));
+                ++use[pb];
+                if (++pb == C::kPBufs) pb = 0;
+#pragma unroll
+                for (int i = 0; i < kSx; ++i) sx[i] = sxn[i];
+                sw0 = sw0n;
+                sw1 = sw1n;
+            }
+            if (!ok) break;
+            const int f = t.m0 + 32 * q + lane;
+            if constexpr (MODE == kGated) {
+                // h = silu(gate) * up, then e4m3 per (token, these 128 features):
+                // the 128 features of a token column are the 4 warps of this half
+                float* red = red_half + (tiles_done & 1u) * 4 * kC;
+#pragma unroll
+                for (int j = 0; j < kC; ++j) {
+                    acc0[j] = silu_mul(acc0[j], acc1[j]);
+                    float m = fabsf(acc0[j]);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    if (lane == 0) red[q * kC + j] = m;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&half_bar[part]));
+                ok = mbar_wait(smem_u32(&half_bar[part]), tiles_done & 1u, abort_flag, p.err);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int j = 0; j < kC; ++j) {
+                    const int col = c_begin + j;
+                    const float amax = fmaxf(fmaxf(red[j], red[kC + j]), fmaxf(red[2 * kC + j], red[3 * kC + j]));
+                    const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+                    if (col < t.n_rows) {
+                        const float v = fminf(fmaxf(acc0[j] / sc, -448.0f), 448.0f);
+                        p.out8[(int64_t)(t.row0 + col) * p.ld_out + f] =
+                            (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+                        if (q == 0 && lane == 0)
+                            p.out_scale[(int64_t)(t.m0 / kBM) * p.act_scale_ld + t.row0 + col] = sc;
+                    }
+                }
+                // red is double buffered by tile parity: the next write of this
+                // buffer comes after every warp of the half has passed the next
+                // tile's barrier, i.e. finished reading it here
+                ++tiles_done;
+            } else {
+#pragma unroll
+                for (int j = 0; j < kC; ++j) {
+                    const int col = c_begin + j;
+                    if (col < t.n_rows) {
+                        __nv_bfloat16* o = p.out + (int64_t)(t.row0 + col) * p.ld_out + f;
+                        o[0] = __float2bfloat16_rn(acc0[j]);
+                        o[kBM] = __float2bfloat16_rn(acc1[j]);
+                    }
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {  // let copies still in flight land before TMEM is released
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 template <int BN, int MODE, bool W8>
 moe_status launch(const FfnArgs& a, int rows, int G, cudaStream_t s) {
@@ -472,6 +794,34 @@ moe_status launch_bn(int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) 
     }
 }
 
+template <int BN, int MODE>
+moe_status launch_f8(const FfnArgs& a, int rows, int G, cudaStream_t s) {
+    using C = CfgF8<BN, MODE>;
+    int sms = 0;
+    moe_status st = sm_count(&sms);
+    if (st != MOE_OK) return st;
+    const int64_t mt = a.M / C::kRowsPerTile;
+    const int64_t bound = mt * ((rows + 15) / 16 + G);
+    const int grid = (int)(bound < sms ? bound : sms);
+    if (grid <= 0) return MOE_OK;
+    auto kern = k_grouped_ffn_f8<BN, MODE>;
+    SWB_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)C::kDynSmem));
+    kern<<<grid, C::kThreads, C::kDynSmem, s>>>(a);
+    SWB_LAUNCHED(MODE == kGated ? "moe_grouped_ffn: fp8 gate/up kernel" : "moe_grouped_ffn: fp8 down kernel");
+    return MOE_OK;
+}
+
+template <int MODE>
+moe_status launch_f8_bn(int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) {
+    switch (bn) {
+        case 16: return launch_f8<16, MODE>(a, rows, G, s);
+        case 32: return launch_f8<32, MODE>(a, rows, G, s);
+        case 64: return launch_f8<64, MODE>(a, rows, G, s);
+        default: return launch_f8<128, MODE>(a, rows, G, s);
+    }
+}
+
 template <int MODE>
 moe_status launch_w(bool w8, int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) {
     return w8 ? launch_bn<MODE, true>(bn, a, rows, G, s) : launch_bn<MODE, false>(bn, a, rows, G, s);
@@ -490,14 +840,25 @@ int pick_bn(int64_t A, int E) {
 // 3-D map {K, rows, slot} over one pool of expert images.  bf16 weights are
 // loaded straight into the MMA operand layout (128-byte swizzle); e4m3
 // weights as plain 64-byte rows for the converter warps.
+// The e4m3 map for the tensor-core fp8 path (f8mma) loads 128-byte rows
+// straight into the MMA operand layout.
 moe_status encode_weight_map(CUtensorMap* m, const void* base, int64_t offset, int32_t count,
-                             int64_t stride, int32_t K, int32_t rows, bool w8) {
+                             int64_t stride, int32_t K, int32_t rows, bool w8, bool f8mma = false) {
     const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)count};
     const uint64_t strides[2] = {(uint64_t)K * (w8 ? 1 : 2), (uint64_t)stride};
-    const uint32_t box[3] = {(uint32_t)kBK, (uint32_t)kBM, 1u};
+    const uint32_t box[3] = {(uint32_t)(f8mma ? 128 : kBK), (uint32_t)kBM, 1u};
     return encode_tiled(m, w8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                         const_cast<char*>(static_cast<const char*>(base)) + offset, dims, strides,
-                        box, w8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+                        box, (w8 && !f8mma) ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+moe_status encode_act_map8(CUtensorMap* m, const void* base, int64_t rows, int32_t K,
+                           uint32_t box_rows) {
+    const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
+    const uint64_t strides[1] = {(uint64_t)K};
+    const uint32_t box[2] = {128u, box_rows};
+    return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 moe_status encode_act_map(CUtensorMap* m, const void* base, int64_t rows, int32_t K,
@@ -515,7 +876,10 @@ moe_status validate(const moe_ffn_desc* d, const moe_expert_table* tb, moe_exper
         d->H <= 0 || d->I <= 0 || d->H % 128 || d->I % 128)
         return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: T=%d H=%d I=%d E=%d k=%d", d->T, d->H,
                     d->I, d->E, d->k);
-    if ((d->w_dtype != MOE_BF16 && d->w_dtype != MOE_E4M3) || d->act_dtype != MOE_BF16)
+    const bool ok_types = (d->w_dtype == MOE_BF16 && d->act_dtype == MOE_BF16) ||
+                          (d->w_dtype == MOE_E4M3 && d->act_dtype == MOE_BF16) ||
+                          (d->w_dtype == MOE_E4M3 && d->act_dtype == MOE_E4M3 && d->H % 256 == 0);
+    if (!ok_types)
         return fail(MOE_ERR_UNSUPPORTED, "moe_grouped_ffn: weight dtype %d / activation dtype %d",
                     d->w_dtype, d->act_dtype);
     moe_status st = moe_expert_layout_get(d->H, d->I, (moe_dtype)d->w_dtype, lay);
@@ -548,6 +912,61 @@ moe_status validate(const moe_ffn_desc* d, const moe_expert_table* tb, moe_exper
     return MOE_OK;
 }
 
+// Both GEMMs on the e4m3 tensor-core path: x_perm and h are e4m3 with
+// per-(row, 128 columns) scales stored [K/128][rows].
+moe_status ffn_f8(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_expert_layout& lay,
+                  const void* x_perm, const float* x_scales, void* h, void* y_perm, float* h_scales,
+                  int rows, int G, FfnArgs& a, cudaStream_t stream) {
+    moe_status st;
+    const void* base[2] = {tbl->local_base, tbl->remote_base};
+    const int32_t count[2] = {tbl->local_count, tbl->remote_count};
+    const int64_t stride[2] = {tbl->local_stride, tbl->remote_stride};
+    int bn = pick_bn(a.A, d->E);
+    if (bn > 128) bn = 128;
+    // GEMM1 -> h (e4m3) and its scales
+    for (int q = 0; q < 2; ++q)
+        if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.gu_offset, count[q],
+                                                    stride[q], d->H, 2 * d->I, true, true)) != MOE_OK)
+            return st;
+    if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.gu_offset, 1,
+                                                 lay.bytes, d->H, 2 * d->I, true, true)) != MOE_OK)
+        return st;
+    if ((st = encode_act_map8(&a.act_map, x_perm, rows, d->H, kBoxN)) != MOE_OK) return st;
+    if ((st = encode_act_map8(&a.act_map64, x_perm, rows, d->H, 64)) != MOE_OK) return st;
+    a.K = d->H;
+    a.M = d->I;
+    a.up_row = d->I;
+    a.ld_out = d->I;
+    a.scale_off = lay.gu_scale_offset;
+    a.kblocks = d->H / 128;
+    a.act_scale = x_scales;
+    a.act_scale_ld = rows;
+    a.out8 = static_cast<uint8_t*>(h);
+    a.out_scale = h_scales;
+    if ((st = launch_f8_bn<kGated>(bn, a, rows, G, stream)) != MOE_OK) return st;
+    // GEMM2 -> y_perm (bf16)
+    for (int q = 0; q < 2; ++q)
+        if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.down_offset,
+                                                    count[q], stride[q], d->I, d->H, true, true)) != MOE_OK)
+            return st;
+    if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.down_offset, 1,
+                                                 lay.bytes, d->I, d->H, true, true)) != MOE_OK)
+        return st;
+    if ((st = encode_act_map8(&a.act_map, h, rows, d->I, kBoxN)) != MOE_OK) return st;
+    if ((st = encode_act_map8(&a.act_map64, h, rows, d->I, 64)) != MOE_OK) return st;
+    a.K = d->I;
+    a.M = d->H;
+    a.up_row = 0;
+    a.ld_out = d->H;
+    a.scale_off = lay.down_scale_offset;
+    a.kblocks = d->I / 128;
+    a.act_scale = h_scales;
+    a.out = static_cast<__nv_bfloat16*>(y_perm);
+    a.out8 = nullptr;
+    a.out_scale = nullptr;
+    return launch_f8_bn<kPair>(bn, a, rows, G, stream);
+}
+
 }  // namespace
 }  // namespace swb
 
@@ -556,17 +975,16 @@ using namespace swb;
 extern "C" {
 
 size_t moe_grouped_ffn_workspace_size(const moe_ffn_desc* d) {
-    (void)d;
-    return 0;
+    // e4m3 activations: the fp32 scales of the e4m3 intermediate h, [I/128][rows]
+    if (!d || d->act_dtype != MOE_E4M3 || d->T <= 0 || d->k <= 0 || d->I <= 0) return 0;
+    const int64_t rows = (int64_t)d->T * d->k + (d->has_shared ? d->T : 0);
+    return (size_t)((d->I / 128) * rows * 4 + 255) / 256 * 256;
 }
 
 moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, const void* x_perm,
                            const float* x_perm_scales, const int32_t* offsets, void* h,
                            void* y_perm, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream) {
-    (void)x_perm_scales;
-    (void)workspace;
-    (void)workspace_bytes;
     moe_expert_layout lay;
     moe_status st = validate(d, tbl, &lay);
     if (st != MOE_OK) return st;
@@ -579,6 +997,15 @@ moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, c
     const int64_t rows = A + (d->has_shared ? d->T : 0);
     if (rows > INT32_MAX / 2) return fail(MOE_ERR_UNSUPPORTED, "moe_grouped_ffn: too many rows");
     const int G = d->E + (d->has_shared ? 1 : 0);
+    const bool f8 = d->act_dtype == MOE_E4M3;
+    if (f8) {
+        const size_t need = moe_grouped_ffn_workspace_size(d);
+        if (!x_perm_scales || !aligned(x_perm_scales, 16))
+            return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: e4m3 activations need x_perm_scales");
+        if (workspace_bytes < need || !workspace || !aligned(workspace, 16))
+            return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn: workspace %zu < %zu bytes",
+                        workspace_bytes, need);
+    }
     int* err = nullptr;
     st = device_error_word(&err);
     if (st != MOE_OK) return st;
@@ -603,6 +1030,8 @@ moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, c
     a.w_stride[0] = tbl->local_stride;
     a.w_stride[1] = tbl->remote_stride;
     a.w_stride[2] = lay.bytes;
+    if (f8) return ffn_f8(d, tbl, lay, x_perm, x_perm_scales, h, y_perm,
+                          static_cast<float*>(workspace), (int)rows, G, a, stream);
 
     // GEMM1: h = silu(X W_gate^T) * (X W_up^T)
     for (int q = 0; q < 2; ++q)

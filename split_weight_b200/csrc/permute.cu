@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(256) k_gather_e4m3(const XT* __restrict__ x,
             packed |= (uint32_t)__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3) << (8 * i);
         }
         *reinterpret_cast<uint32_t*>(out + r * H + c0 + lane * 4) = packed;
-        if (lane == 0) scales[r * (H / 128) + c0 / 128] = s;
+        if (lane == 0) scales[(int64_t)(c0 / 128) * rows + r] = s;  // [H/128][rows]
     }
 }
 

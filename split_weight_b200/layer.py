@@ -44,6 +44,9 @@ class LayerShape:
     x_dtype: str = "bf16"        # "f32" | "bf16"
     w_dtype: str = "bf16"        # "bf16" | "e4m3"
     y_dtype: str = "bf16"        # "f32" | "bf16"
+    # activations the grouped GEMMs read: "bf16", or "e4m3" (with e4m3 weights:
+    # both GEMMs on the fp8 tensor cores, x_perm and h e4m3 with 1x128 scales)
+    act_dtype: str = "bf16"
 
     @property
     def A(self) -> int:
@@ -61,7 +64,7 @@ class LayerShape:
 
     def ffn_desc(self) -> L.moe_ffn_desc:
         return L.moe_ffn_desc(self.T, self.H, self.I, self.E, self.k, _DT[self.w_dtype],
-                              L.MOE_BF16, 1 if self.has_shared else 0)
+                              _DT[self.act_dtype], 1 if self.has_shared else 0)
 
 
 def _stream_handle(stream: torch.cuda.Stream | None) -> int:
@@ -145,8 +148,13 @@ class MoELayer:
         self.perm_src = torch.empty(max(s.A, 1), dtype=i32, device=dev)
         self.inv_pos = torch.empty(max(s.T, 1), s.k, dtype=i32, device=dev)
         rows = max(s.rows, 1)
-        self.x_perm = torch.empty(rows, s.H, dtype=torch.bfloat16, device=dev)
-        self.h = torch.empty(rows, s.I, dtype=torch.bfloat16, device=dev)
+        a8 = s.act_dtype == "e4m3"
+        adt = torch.uint8 if a8 else torch.bfloat16
+        self.x_perm = torch.empty(rows, s.H, dtype=adt, device=dev)
+        self.x_scales = torch.empty(s.H // 128, rows, dtype=torch.float32, device=dev) if a8 else None
+        self.h = torch.empty(rows, s.I, dtype=adt, device=dev)
+        self.ffn_ws = torch.empty(max(L.moe_grouped_ffn_workspace_size(ctypes.byref(self._desc)), 16),
+                                  dtype=torch.uint8, device=dev)
         self.y_perm = torch.empty(rows, s.H, dtype=torch.bfloat16, device=dev)
         ydt = torch.float32 if s.y_dtype == "f32" else torch.bfloat16
         self.y = torch.empty(max(s.T, 1), s.H, dtype=ydt, device=dev)
@@ -161,16 +169,19 @@ class MoELayer:
     def permute(self, x: torch.Tensor, stream: int) -> None:
         s = self.shape
         L.check(L.moe_permute(s.T, s.k, s.E, s.H, self.topk_idx.data_ptr(), x.data_ptr(),
-                              _DT[s.x_dtype], L.MOE_BF16, 1 if s.has_shared else 0,
+                              _DT[s.x_dtype], _DT[s.act_dtype], 1 if s.has_shared else 0,
                               self.offsets.data_ptr(), self.perm_src.data_ptr(),
-                              self.inv_pos.data_ptr(), self.x_perm.data_ptr(), None,
+                              self.inv_pos.data_ptr(), self.x_perm.data_ptr(),
+                              _ptr(self.x_scales),
                               self.perm_ws.data_ptr(), self.perm_ws.numel(), stream))
 
     def grouped_ffn(self, stream: int, remote: torch.Tensor | None = None) -> None:
         tbl = self.weights.table(remote)
         L.check(L.moe_grouped_ffn(ctypes.byref(self._desc), ctypes.byref(tbl),
-                                  self.x_perm.data_ptr(), None, self.offsets.data_ptr(),
-                                  self.h.data_ptr(), self.y_perm.data_ptr(), None, 0, stream))
+                                  self.x_perm.data_ptr(), _ptr(self.x_scales),
+                                  self.offsets.data_ptr(), self.h.data_ptr(),
+                                  self.y_perm.data_ptr(), self.ffn_ws.data_ptr(),
+                                  self.ffn_ws.numel(), stream))
 
     def combine(self, stream: int) -> None:
         s = self.shape

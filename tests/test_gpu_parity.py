@@ -48,6 +48,8 @@ def _check_permutation(dl, idx_ref):
     np.testing.assert_array_equal(ml.offsets.cpu().numpy(), off)
     np.testing.assert_array_equal(ml.perm_src[:c.A].cpu().numpy(), src)
     np.testing.assert_array_equal(ml.inv_pos[:c.T].cpu().numpy(), inv)
+    if ml.shape.act_dtype != "bf16":
+        return   # e4m3 rows: see test_e4m3_gather_quantises_each_128_block
     # gathered rows: x (rounded to bf16 when it came as fp32), then the shared rows
     xp = ml.x_perm[:c.rows].view(torch.int16).cpu().numpy().view(np.uint16)
     xb = gen.f32_to_bf16_bits(dl.inputs.x)
@@ -68,6 +70,18 @@ def test_small_layer_full_parity(cfg):
     _check_routing(dl, idx_ref, w_ref)
     _check_permutation(dl, idx_ref)
     assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
+
+
+@pytest.mark.parametrize("cfg", [MID_FP8, DECODE_FP8], ids=lambda c: c.name)
+def test_fp8_weights_with_bf16_activations(cfg):
+    """The conversion path: e4m3 weights dequantised to bf16 in shared memory,
+    bf16 activations, bf16 tensor-core MMA."""
+    dl = mdev.build_layer(cfg, act_dtype="bf16")
+    run_layer(dl)
+    y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
+    _check_routing(dl, idx_ref, w_ref)
+    _check_permutation(dl, idx_ref)
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, RTOL_FP8, f"{cfg.name} y (bf16 act)")
 
 
 def test_generator_gpu_matches_host(cuda_device):
@@ -191,7 +205,7 @@ def test_e4m3_gather_quantises_each_128_block(cuda_device):
     src = torch.empty(T * k, dtype=torch.int32, device=dev)
     inv = torch.empty(T, k, dtype=torch.int32, device=dev)
     xq = torch.empty(rows, H, dtype=torch.uint8, device=dev)
-    sc = torch.empty(rows, H // 128, dtype=torch.float32, device=dev)
+    sc = torch.empty(H // 128, rows, dtype=torch.float32, device=dev)   # [H/128, rows]
     ws = torch.empty(L.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=dev)
     L.check(L.moe_permute(T, k, E, H, idx.data_ptr(), x.data_ptr(), L.MOE_BF16, L.MOE_E4M3, 1,
                           off.data_ptr(), src.data_ptr(), inv.data_ptr(), xq.data_ptr(),
@@ -201,12 +215,13 @@ def test_e4m3_gather_quantises_each_128_block(cuda_device):
     o_ref, s_ref, _ = oracle.permute(idx_ref, E)
     np.testing.assert_array_equal(src.cpu().numpy(), s_ref)
     xs = np.concatenate([li.x[s_ref], li.x]).astype(np.float64)
-    dec = gen.e4m3_bits_to_f64(xq.cpu().numpy()) * np.repeat(sc.cpu().numpy(), 128, axis=1)
+    scr = sc.cpu().numpy().T                                  # [rows, H/128]
+    dec = gen.e4m3_bits_to_f64(xq.cpu().numpy()) * np.repeat(scr, 128, axis=1)
     blk = np.abs(xs).reshape(rows, H // 128, 128).max(axis=2)
-    np.testing.assert_allclose(sc.cpu().numpy(), blk / 448, rtol=1e-6)
+    np.testing.assert_allclose(scr, blk / 448, rtol=1e-6)
     # e4m3 has 3 mantissa bits: |err| <= 2^-4 |v| for normal codes, plus the
     # subnormal step 2^-10 * s
-    bound = np.abs(xs) * 2.0 ** -4 + np.repeat(sc.cpu().numpy(), 128, axis=1) * 2.0 ** -10
+    bound = np.abs(xs) * 2.0 ** -4 + np.repeat(scr, 128, axis=1) * 2.0 ** -10
     assert (np.abs(dec - xs) <= bound * (1 + 1e-6)).all()
 
 
