@@ -123,7 +123,7 @@ struct CfgF8 {
     static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024 + kScratch;
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                   "TMEM allocation must be a power of two in [32, 512]");
-    static_assert(kStages >= 2 && BN <= 128 && BN % 16 == 0, "fp8 tile shape");
+    static_assert(kStages >= 2 && BN <= 64 && BN % 16 == 0, "fp8 tile shape");
 };
 
 struct Tile {
@@ -672,27 +672,28 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t tp = tmem_base + ((uint32_t)(32 * q) << 16) + pb * C::kPartCols + c_begin;
-#pragma unroll
-                for (int c0 = 0; c0 < kC; c0 += 8) {
-                    float a[8], b[8];
-                    tmem_ld_8(tp + c0, a);
-                    tmem_ld_8(tp + BN + c0, b);
-                    tmem_ld_wait();
-                    const float4 g0 = *reinterpret_cast<const float4*>(cg + c0);
-                    const float4 g1 = *reinterpret_cast<const float4*>(cg + c0 + 4);
-                    const float4 u0 = *reinterpret_cast<const float4*>(cu + c0);
-                    const float4 u1 = *reinterpret_cast<const float4*>(cu + c0 + 4);
-                    const float gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                    const float us[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        acc0[c0 + i] = fmaf(a[i], gs[i], acc0[c0 + i]);
-                        acc1[c0 + i] = fmaf(b[i], us[i], acc1[c0 + i]);
-                    }
-                }
+                // the warp's whole slice of both partial sums, one wait, then the
+                // buffer goes straight back to the MMA
+                float a[kC], b[kC];
+                tmem_ld_n<kC>(tp, a);
+                tmem_ld_n<kC>(tp + BN, b);
+                tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&part_empty[pb]));
+#pragma unroll
+                for (int c0 = 0; c0 < kC; c0 += 4) {
+                    const float4 g = *reinterpret_cast<const float4*>(cg + c0);
+                    const float4 u = *reinterpret_cast<const float4*>(cu + c0);
+                    acc0[c0] = fmaf(a[c0], g.x, acc0[c0]);
+                    acc0[c0 + 1] = fmaf(a[c0 + 1], g.y, acc0[c0 + 1]);
+                    acc0[c0 + 2] = fmaf(a[c0 + 2], g.z, acc0[c0 + 2]);
+                    acc0[c0 + 3] = fmaf(a[c0 + 3], g.w, acc0[c0 + 3]);
+                    acc1[c0] = fmaf(b[c0], u.x, acc1[c0]);
+                    acc1[c0 + 1] = fmaf(b[c0 + 1], u.y, acc1[c0 + 1]);
+                    acc1[c0 + 2] = fmaf(b[c0 + 2], u.z, acc1[c0 + 2]);
+                    acc1[c0 + 3] = fmaf(b[c0 + 3], u.w, acc1[c0 + 3]);
+                }
                 ++use[pb];
                 if (++pb == C::kPBufs) pb = 0;
 #pragma unroll
@@ -817,8 +818,7 @@ moe_status launch_f8_bn(int bn, const FfnArgs& a, int rows, int G, cudaStream_t 
     switch (bn) {
         case 16: return launch_f8<16, MODE>(a, rows, G, s);
         case 32: return launch_f8<32, MODE>(a, rows, G, s);
-        case 64: return launch_f8<64, MODE>(a, rows, G, s);
-        default: return launch_f8<128, MODE>(a, rows, G, s);
+        default: return launch_f8<64, MODE>(a, rows, G, s);
     }
 }
 
@@ -921,8 +921,10 @@ moe_status ffn_f8(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_
     const void* base[2] = {tbl->local_base, tbl->remote_base};
     const int32_t count[2] = {tbl->local_count, tbl->remote_count};
     const int64_t stride[2] = {tbl->local_stride, tbl->remote_stride};
+    // token tiles of at most 64: a warp then folds its 32 columns of both
+    // partial sums with one TMEM read, and 4 partial buffers let the MMA run ahead
     int bn = pick_bn(a.A, d->E);
-    if (bn > 128) bn = 128;
+    if (bn > 64) bn = 64;
     // GEMM1 -> h (e4m3) and its scales
     for (int q = 0; q < 2; ++q)
         if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.gu_offset, count[q],
