@@ -35,7 +35,6 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s at DeepSeek-R1 shape; % of HBM/tensor roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_LAYER = 9  # route 2 + permute 4 + grouped FFN 2 + combine 1
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "grouped_ffn_traffic.json")
 
 
@@ -48,6 +47,7 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-merge-ablation", action="store_true")
     return p.parse_args(argv)
 
 
@@ -62,26 +62,36 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
     h = hashlib.sha256()
-    for name in ("ffn.cu", "device.cuh"):
+    for name in files:
         with open(os.path.join(ROOT, "split_weight_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the grouped FFN from the committed ncu
-    summary, if it was taken on the current kernel source."""
+def profiled_traffic(workload: str, alg_bytes_per_layer: float):
+    """DRAM bytes per layer of the grouped FFN (gate/up + down launches) from
+    the committed ncu capture, if it was taken on the current kernel source.
+    A full-size workload too large to capture is scaled from its reduced
+    case by the ratio of algorithmic bytes (same tokens per expert)."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
     e = d.get(workload)
-    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+    if not e:
         return None
-    return e.get("dram_bytes_per_call")
+    scale = 1.0
+    if "scaled_from" in e:
+        e = d.get(e["scaled_from"])
+        if not e:
+            return None
+        scale = alg_bytes_per_layer / e["algorithmic_bytes_per_call"]
+    if e.get("kernel_source_hash") != kernel_source_hash(e["kernel_files"]):
+        return None
+    return e["dram_bytes_per_call"] * scale
 
 
 class ClockSampler:
@@ -247,10 +257,12 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
+        launches0 = L.moe_kernel_launches()
         ev0.record(stream)
         for i in range(args.steps):
             step(ffn_ev[i])
         ev1.record(stream)
+        launches = L.moe_kernel_launches() - launches0
         torch.cuda.synchronize()
     elapsed_ms = ev0.elapsed_time(ev1)
     ffn_ms = sum(a.elapsed_time(b) for st in ffn_ev for a, b in st) / args.steps
@@ -289,6 +301,12 @@ def run_ours(args, rank, world, local_rank):
             "exposed_copy_ms_per_layer": round(exposed, 4),
             "hidden_fraction": round(1.0 - exposed / copy_ms, 4) if copy_ms > 0 else None,
         }
+
+    # ---- split-weight ablation: merge both pools into one buffer every step
+    merge_info = None
+    if pipe is None and not args.no_merge_ablation:
+        merge_info = merge_ablation(cfg, dls[0], stream, elapsed_ms / args.steps,
+                                    max(3, min(args.steps, 20)))
 
     # ---- end-to-end through the public API with host buffers
     e2e = None
@@ -346,9 +364,9 @@ def run_ours(args, rank, world, local_rank):
         achieved = flops / ffn_s / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4)}
-    traffic = profiled_traffic(workload)
+    traffic = profiled_traffic(workload, nbytes / cfg.layers)
     roof.update({
-        "traffic": (traffic * cfg.layers if traffic is not None else None),
+        "traffic": (round(traffic * cfg.layers) if traffic is not None else None),
         "kernel": "moe_grouped_ffn (gate/up + down launches)",
         "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
         "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
@@ -368,12 +386,68 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2: %.1f GB of expert weights per step" % (nbytes / 1e9)},
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": LAUNCHES_PER_LAYER * cfg.layers * args.steps,
+        "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    if merge_info is not None:
+        out["split_weight"] = merge_info
     if prefetch_info is not None:
         out["prefetch"] = prefetch_info
     return out, cfg
+
+
+def merge_ablation(cfg, dl, stream, split_step_ms: float, reps: int):
+    """The alternative the explainer's split-weight figure argues against: copy
+    the local and the remote experts into one contiguous buffer (expert order)
+    before every grouped GEMM, then address it as a single pool.  Returns the
+    merge copy time and the step time with it, next to the split-table step."""
+    import numpy as np
+    import torch
+    from split_weight_b200 import SplitWeights
+    from split_weight_b200 import _lib as L
+    ml = dl.layer
+    w = ml.weights
+    merged = torch.empty(cfg.E * w.stride, dtype=torch.uint8, device=w.local.device)
+    h = stream.cuda_stream
+
+    def merge():
+        # the default placement keeps experts in slot order in each pool:
+        # local = experts [0, n_local), remote = the rest
+        L.check(L.moe_prefetch_layer(w.local.data_ptr(), merged.data_ptr(), w.n_local * w.stride,
+                                     0, h, None, None))
+        L.check(L.moe_prefetch_layer(w.remote.data_ptr(), merged.data_ptr() + w.n_local * w.stride,
+                                     w.n_remote * w.stride, 0, h, None, None))
+
+    ps = np.arange(cfg.E, dtype=np.int64)
+    mw = SplitWeights(w.H, w.I, w.w_dtype, ps.astype(np.int32), merged, cfg.E, merged[:1], 0,
+                      w.shared)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    merge()
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(reps):
+        merge()
+    ev[1].record(stream)
+    saved = ml.weights
+    ml.weights = mw
+    try:
+        ev[2].record(stream)
+        for _ in range(reps):
+            merge()
+            ml.route(dl.x, h)
+            ml.permute(dl.x, h)
+            ml.grouped_ffn(h)
+            ml.combine(h)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+    finally:
+        ml.weights = saved
+    merge_ms = ev[0].elapsed_time(ev[1]) / reps
+    merged_step = ev[2].elapsed_time(ev[3]) / reps
+    return {"merged_buffer_bytes": cfg.E * w.stride, "merge_copy_ms": round(merge_ms, 4),
+            "step_ms_split_table": round(split_step_ms, 4),
+            "step_ms_merge_then_gemm": round(merged_step, 4),
+            "merge_overhead_fraction": round(merged_step / split_step_ms - 1.0, 4)}
 
 
 # ----------------------------------------------------------------------- oracle

@@ -77,6 +77,11 @@ MOE_API const char *moe_status_string(moe_status s);
 MOE_API const char *moe_last_error(void);
 /* MOE_ABI_VERSION of the loaded library. */
 MOE_API int32_t moe_abi_version(void);
+/* Number of kernels this library has launched in this process (all threads,
+ * all devices), counted after each launch the runtime accepted.  Copies
+ * issued by moe_prefetch_layer are not kernels and are not counted.  A
+ * caller takes the difference of two readings around a region of calls. */
+MOE_API uint64_t moe_kernel_launches(void);
 
 /* ------------------------------------------------------------------------
  * Routing: router logits, scores and top-k selection.

@@ -61,6 +61,7 @@ _SIGS = {
     "moe_status_string": ([i32], ctypes.c_char_p),
     "moe_last_error": ([], ctypes.c_char_p),
     "moe_abi_version": ([], i32),
+    "moe_kernel_launches": ([], ctypes.c_uint64),
     "moe_route_workspace_size": ([ctypes.POINTER(moe_route_cfg)], sz),
     "moe_route": ([ctypes.POINTER(moe_route_cfg), vp, i32, vp, vp, vp, vp, vp, sz, vp], i32),
     "moe_permute_workspace_size": ([i32, i32, i32], sz),
@@ -104,6 +105,7 @@ def check(status: int) -> None:
 
 
 moe_abi_version = _lib.moe_abi_version
+moe_kernel_launches = _lib.moe_kernel_launches
 moe_route_workspace_size = _lib.moe_route_workspace_size
 moe_route = _lib.moe_route
 moe_permute_workspace_size = _lib.moe_permute_workspace_size

@@ -109,6 +109,9 @@ moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t ra
     return MOE_OK;
 }
 
+std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 }  // namespace swb
 
 using namespace swb;
@@ -131,6 +134,8 @@ const char* moe_status_string(moe_status s) {
 const char* moe_last_error(void) { return g_last_error; }
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 void moe_debug_fail_next_cuda_calls(int32_t count) { g_fail_next.store(count > 0 ? count : 0); }
 

@@ -1,0 +1,303 @@
+// The bf16 tensor-core grouped FFN kernel (kind::f16), with bf16 weights or
+// with e4m3 weights that converter warps dequantise into the staged tiles.
+#pragma once
+
+#include "ffn_common.cuh"
+
+namespace swb {
+namespace {
+
+constexpr uint32_t kA8Bytes = kBM * kBK;       // one e4m3 weight tile as loaded, 8 KB
+constexpr int kConvThreads = 256;              // e4m3 -> bf16 converter warps (8)
+
+// Per stage: the bf16 weight tile(s) the MMA reads (128-byte swizzled), the
+// token tile, and for e4m3 weights the staging tile(s) TMA writes.
+template <int BN, int MODE, bool W8>
+struct Cfg {
+    static constexpr int kNA = MODE == kSingle ? 1 : 2;           // weight tiles per stage
+    static constexpr uint32_t kAStage = kABytes * kNA;
+    static constexpr uint32_t kBStage = BN * kBK * 2;
+    static constexpr uint32_t kA8Stage = W8 ? kA8Bytes * kNA : 0;
+    static constexpr uint32_t kStageBytes = kAStage + kBStage + kA8Stage;
+    static constexpr int kStages = (kSmemBudget / kStageBytes) > 12 ? 12 : (kSmemBudget / kStageBytes);
+    static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
+    static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+    static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
+    static constexpr int kEpiWarps = BN >= 256 ? 8 : 4;
+    static constexpr int kConvWarps = W8 ? kConvThreads / 32 : 0;
+    static constexpr int kConvFirstWarp = 2 + kEpiWarps;
+    static constexpr int kThreads = 64 + 32 * (kEpiWarps + kConvWarps);
+    static constexpr int kRowsPerTile = MODE == kPair ? 2 * kBM : kBM;  // output features
+    static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024;
+    static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                  "TMEM allocation must be a power of two in [32, 512]");
+    static_assert(kStages >= 2, "pipeline needs two stages");
+};
+// 16 e4m3 weights (one 16-byte chunk of a staged row) times their block
+// scale, rounded to bf16: 32 bytes, the two 16-byte chunks that follow.
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 in, float s, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * h));
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * s, f.y * s);
+            o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int BN, int MODE, bool W8>
+__global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
+    k_grouped_ffn(const __grid_constant__ FfnArgs p) {
+    using C = Cfg<BN, MODE, W8>;
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
+    __shared__ __align__(8) uint64_t conv_bar[W8 ? C::kStages : 1];  // bf16 tiles converted
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ Tables tb;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t stages = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    const int G = p.E + (p.has_shared ? 1 : 0);
+    const int MT = p.M / C::kRowsPerTile;
+    const int KB = p.K / kBK;
+    volatile int* abort_flag = &abort_sh;
+
+    if (threadIdx.x == 0) {
+        abort_sh = 0;
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+            if constexpr (W8) mbar_init(smem_u32(&conv_bar[s]), C::kConvWarps);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&acc_full[a]), 1);
+            mbar_init(smem_u32(&acc_empty[a]), C::kEpiWarps);
+        }
+        fence_mbar_init();
+        tma_prefetch_map(&p.act_map);
+        tma_prefetch_map(&p.act_map64);
+        for (int m = 0; m < 3; ++m) tma_prefetch_map(&p.w_map[m]);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 2) build_tables<BN>(p, tb, G, MT, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+    const int total = tb.tile_start[G];
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+                const CUtensorMap* wm = &p.w_map[t.map];
+                const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
+                const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const uint32_t eb = smem_u32(&empty_bar[stage]);
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    if (!mbar_wait(eb, phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    mbar_arrive_expect_tx(fb, tx);
+                    // e4m3 weights land in the staging area, bf16 ones straight in the operand
+                    const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
+                    const uint32_t w_step = W8 ? kA8Bytes : kABytes;
+                    tma_load_3d(sw, wm, fb, kb * kBK, t.m0, t.slot);
+                    if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * kBK, row_a1, t.slot);
+                    const uint32_t sb = sa + C::kAStage;
+                    int r = 0;
+                    for (; r + 64 <= t.n_mma; r += 64)
+                        tma_load_2d(sb + r * kBK * 2, &p.act_map64, fb, kb * kBK, t.row0 + r);
+                    for (; r < t.n_mma; r += kBoxN)
+                        tma_load_2d(sb + r * kBK * 2, &p.act_map, fb, kb * kBK, t.row0 + r);
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_use[2] = {0u, 0u};
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+                if (!mbar_wait(smem_u32(&acc_empty[acc]), (acc_use[acc] & 1u) ^ 1u, abort_flag,
+                               p.err))
+                    break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * C::kAccCols;
+                const uint32_t idesc = idesc_bf16_f32(kBM, t.n_mma);
+                for (int kb = 0; kb < KB; ++kb) {
+                    const uint32_t ready_bar = W8 ? smem_u32(&conv_bar[stage]) : smem_u32(&full_bar[stage]);
+                    if (!mbar_wait(ready_bar, phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    const uint32_t sb = sa + C::kAStage;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint32_t accum = (kb | kk) != 0;
+                        const uint64_t bd = sw128_desc(sb + kk * 32);
+                        mma_bf16_ss(d0, sw128_desc(sa + kk * 32), bd, idesc, accum);
+                        if constexpr (C::kNA == 2)
+                            mma_bf16_ss(d0 + BN, sw128_desc(sa + kABytes + kk * 32), bd, idesc, accum);
+                    }
+                    mma_commit(smem_u32(&empty_bar[stage]));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&acc_full[acc]));
+                ++acc_use[acc];
+                if (C::kAccBufs == 2) acc ^= 1;
+            }
+        }
+    } else if (W8 && warp >= C::kConvFirstWarp) {
+        // ------------------------------------------------ e4m3 -> bf16 converters
+        // Each staged row is 64 e4m3 bytes (4 chunks of 16); the bf16 operand
+        // row is 128 bytes in the 128-byte swizzle: 16-byte chunk j of row r
+        // sits at position j ^ (r % 8).  One 128x128 block scale covers the
+        // whole stage (64 columns of K, 128 rows).
+        const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. kConvThreads-1
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+            const uint8_t* sbase = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map] + p.scale_off;
+            const float* sc0 = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
+            const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
+            const float* sc1 = reinterpret_cast<const float*>(sbase) + (int64_t)rb1 * p.kblocks;
+            for (int kb = 0; kb < KB; ++kb) {
+                const float s0 = __ldg(sc0 + (kb >> 1));
+                const float s1 = C::kNA == 2 ? __ldg(sc1 + (kb >> 1)) : 0.0f;
+                ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = stages + stage * C::kStageBytes;
+                const uint32_t s8 = sa + C::kAStage + C::kBStage;
+#pragma unroll
+                for (int a = 0; a < C::kNA; ++a) {
+                    const float sc = a == 0 ? s0 : s1;
+#pragma unroll
+                    for (int i = 0; i < (kBM * kBK / 16) / kConvThreads; ++i) {
+                        const int id = ct + kConvThreads * i, r = id >> 2, c = id & 3;
+                        uint4 in, lo, hi;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(in.x), "=r"(in.y), "=r"(in.z), "=r"(in.w)
+                                     : "r"(s8 + a * kA8Bytes + r * kBK + c * 16));
+                        e4m3x16_to_bf16(in, sc, lo, hi);
+                        const uint32_t row = sa + a * kABytes + r * 128;
+                        const uint32_t j0 = (2 * c) ^ (r & 7), j1 = (2 * c + 1) ^ (r & 7);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j0 * 16),
+                                     "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
+                                     : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j1 * 16),
+                                     "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                                     : "memory");
+                    }
+                }
+                // generic-proxy stores -> visible to the tensor core's async proxy
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&conv_bar[stage]));
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;                    // TMEM lane quarter this warp may access
+        const int part = (warp - 2) >> 2;          // column half (8 epilogue warps) or 0
+        constexpr int kCols = C::kEpiWarps == 8 ? BN / 2 : BN;
+        int acc = 0;
+        uint32_t acc_use[2] = {0u, 0u};
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+            bool ok = mbar_wait(smem_u32(&acc_full[acc]), acc_use[acc] & 1u, abort_flag, p.err);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + ((uint32_t)(32 * q) << 16) + acc * C::kAccCols;
+            const int f = t.m0 + 32 * q + lane;
+            __nv_bfloat16* out = p.out + (int64_t)t.row0 * p.ld_out + f;
+            const int c_begin = part * kCols, c_end = min(t.n_rows, c_begin + kCols);
+            for (int c0 = c_begin; c0 < c_end; c0 += 16) {
+                float g[16];
+                tmem_ld_16(tacc + c0, g);
+                if constexpr (C::kNA == 2) {
+                    float u[16];
+                    tmem_ld_16(tacc + BN + c0, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (c0 + i >= t.n_rows) continue;
+                        __nv_bfloat16* o = out + (int64_t)(c0 + i) * p.ld_out;
+                        if constexpr (MODE == kGated) {
+                            o[0] = __float2bfloat16_rn(silu_mul(g[i], u[i]));
+                        } else {
+                            o[0] = __float2bfloat16_rn(g[i]);
+                            o[kBM] = __float2bfloat16_rn(u[i]);
+                        }
+                    }
+                } else {
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < t.n_rows)
+                            out[(int64_t)(c0 + i) * p.ld_out] = __float2bfloat16_rn(g[i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+            ++acc_use[acc];
+            if (C::kAccBufs == 2) acc ^= 1;
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {  // let copies still in flight land before TMEM is released
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+}  // namespace
+}  // namespace swb

@@ -28,11 +28,15 @@ moe_status cuda_check(cudaError_t e, const char* what);
         if (_e != cudaSuccess) return ::swb::cuda_check(_e, #call);             \
     } while (0)
 
-// After a launch: report launch-configuration errors.
+// Counts the kernels the library has launched (process-wide).
+void count_launch();
+
+// After a launch: report launch-configuration errors, count the launch.
 #define SWB_LAUNCHED(what)                                                      \
     do {                                                                        \
         cudaError_t _e = cudaGetLastError();                                    \
         if (_e != cudaSuccess) return ::swb::cuda_check(_e, what);              \
+        ::swb::count_launch();                                                  \
     } while (0)
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

@@ -20,57 +20,108 @@ namespace {
 constexpr int kChunk = 256;  // h per fused-multiply-add chain
 constexpr int kKT = 32;      // h per shared-memory tile
 
-__device__ __forceinline__ float load_x(const float* x, int64_t i) { return x[i]; }
-__device__ __forceinline__ float load_x(const __nv_bfloat16* x, int64_t i) {
-    return __bfloat162float(x[i]);
+// Two IEEE fused multiply-adds in one sm_100 instruction (packed fp32):
+// lane i of d becomes fma(a_i, b_i, d_i), rounded to nearest like fmaf.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ void fma2(uint64_t& d, uint64_t a, uint64_t b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+
+// Eight consecutive values as fp32 (16-byte aligned source), or zeros.
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, bool in, float (&r)[8]) {
+    const uint4 u = in ? *reinterpret_cast<const uint4*>(p) : make_uint4(0, 0, 0, 0);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(b2[i]);
+        r[2 * i] = f.x;
+        r[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float* p, bool in, float (&r)[8]) {
+    const float4 a = in ? *reinterpret_cast<const float4*>(p) : make_float4(0, 0, 0, 0);
+    const float4 b = in ? *reinterpret_cast<const float4*>(p + 4) : make_float4(0, 0, 0, 0);
+    r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
+    r[4] = b.x; r[5] = b.y; r[6] = b.z; r[7] = b.w;
 }
 
 // Each thread owns a TM x TN block of (token, expert) pairs of a
-// (16 TM) x (16 TN) block tile.  With split != 0 the z index of the grid is
-// the chunk and the kernel writes that chunk's sum P_c to part[c][t][e];
-// otherwise it walks all chunks and writes l[t][e].
+// (16 TM) x (16 TN) block tile; 32 h per shared-memory stage, the next
+// stage's global loads held in registers while the current one is consumed.
+// With split != 0 the z index of the grid is the chunk and the kernel writes
+// that chunk's sum P_c to part[c][t][e]; otherwise it walks all chunks and
+// writes l[t][e].
 template <typename XT, int TM, int TN>
 __global__ void __launch_bounds__(256) k_logits(const XT* __restrict__ x,
                                                 const float* __restrict__ wg, int T, int H, int E,
                                                 int split, float* __restrict__ out) {
     constexpr int BT = 16 * TM, BE = 16 * TN;
-    __shared__ __align__(16) float xs[kKT][BT + 4];
-    __shared__ __align__(16) float ws[kKT][BE + 4];
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    static_assert(TN % 2 == 0 && BT * kKT / 8 <= 256 && BE * kKT / 8 <= 256, "tile");
+    __shared__ __align__(16) float xs[2][kKT][BT + 4];  // [buffer][h][token]
+    __shared__ __align__(16) float ws[2][kKT][BE + 4];  // [buffer][h][expert]
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int e0 = blockIdx.x * BE, t0 = blockIdx.y * BT;
     int h_begin = 0, h_end = H;
     if (split) {
         h_begin = blockIdx.z * kChunk;
         h_end = min(H, h_begin + kChunk);
     }
-    float l[TM][TN], p[TM][TN];
+    // loader: thread tid moves 8 consecutive h of tile row tid / 4
+    const int lr = tid >> 2, lh = (tid & 3) * 8;
+    const bool xl = tid < BT * kKT / 8, wl = tid < BE * kKT / 8;
+    const bool xin = xl && t0 + lr < T, win = wl && e0 + lr < E;
+    const XT* xrow = x + (int64_t)(xin ? t0 + lr : 0) * H + lh;
+    const float* wrow = wg + (int64_t)(win ? e0 + lr : 0) * H + lh;
+    float rx[8], rw[8];
+    auto store = [&](int buf) {
 #pragma unroll
-    for (int i = 0; i < TM; ++i)
+        for (int i = 0; i < 8; ++i) {
+            if (xl) xs[buf][lh + i][lr] = rx[i];
+            if (wl) ws[buf][lh + i][lr] = rw[i];
+        }
+    };
+    float l[TM][TN];
+    uint64_t p[TM][TN / 2];  // chain sums of columns 2q, 2q + 1
 #pragma unroll
-        for (int j = 0; j < TN; ++j) l[i][j] = p[i][j] = 0.0f;
-
-    for (int h0 = h_begin; h0 < h_end; h0 += kKT) {
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < BT * kKT; idx += 256) {
-            const int tt = idx / kKT, kk = idx % kKT, t = t0 + tt;
-            xs[kk][tt] = (t < T) ? load_x(x, (int64_t)t * H + h0 + kk) : 0.0f;
+    for (int i = 0; i < TM; ++i) {
+#pragma unroll
+        for (int j = 0; j < TN; ++j) l[i][j] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < TN / 2; ++q) p[i][q] = 0;
+    }
+    const int nk = (h_end - h_begin) / kKT;
+    load8(xrow + h_begin, xin, rx);
+    load8(wrow + h_begin, win, rw);
+    store(0);
+    __syncthreads();
+    for (int it = 0; it < nk; ++it) {
+        const int buf = it & 1, h0 = h_begin + it * kKT;
+        if (it + 1 < nk) {
+            load8(xrow + h0 + kKT, xin, rx);
+            load8(wrow + h0 + kKT, win, rw);
         }
-        for (int idx = threadIdx.x; idx < BE * kKT; idx += 256) {
-            const int ee = idx / kKT, kk = idx % kKT, e = e0 + ee;
-            ws[kk][ee] = (e < E) ? wg[(int64_t)e * H + h0 + kk] : 0.0f;
-        }
-        __syncthreads();
 #pragma unroll 8
         for (int kk = 0; kk < kKT; ++kk) {
             float a[TM], b[TN];
 #pragma unroll
-            for (int i = 0; i < TM; ++i) a[i] = xs[kk][ty * TM + i];
+            for (int i = 0; i < TM; ++i) a[i] = xs[buf][kk][ty * TM + i];
 #pragma unroll
-            for (int j = 0; j < TN; ++j) b[j] = ws[kk][tx * TN + j];
+            for (int j = 0; j < TN; ++j) b[j] = ws[buf][kk][tx * TN + j];
 #pragma unroll
-            for (int i = 0; i < TM; ++i)
+            for (int i = 0; i < TM; ++i) {
+                const uint64_t ai = pack2(a[i], a[i]);
 #pragma unroll
-                for (int j = 0; j < TN; ++j) p[i][j] = __fmaf_rn(a[i], b[j], p[i][j]);
+                for (int q = 0; q < TN / 2; ++q) fma2(p[i][q], ai, pack2(b[2 * q], b[2 * q + 1]));
+            }
         }
         const int h_next = h0 + kKT;
         if (h_next % kChunk == 0 || h_next >= h_end) {  // a chunk ends here
@@ -78,11 +129,15 @@ __global__ void __launch_bounds__(256) k_logits(const XT* __restrict__ x,
 #pragma unroll
             for (int i = 0; i < TM; ++i)
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    l[i][j] = first ? p[i][j] : __fadd_rn(l[i][j], p[i][j]);
-                    p[i][j] = 0.0f;
+                for (int q = 0; q < TN / 2; ++q) {
+                    const float2 v = unpack2(p[i][q]);
+                    l[i][2 * q] = first ? v.x : __fadd_rn(l[i][2 * q], v.x);
+                    l[i][2 * q + 1] = first ? v.y : __fadd_rn(l[i][2 * q + 1], v.y);
+                    p[i][q] = 0;
                 }
         }
+        if (it + 1 < nk) store(buf ^ 1);
+        __syncthreads();
     }
     float* o = split ? out + (int64_t)blockIdx.z * T * E : out;
 #pragma unroll
@@ -97,29 +152,30 @@ __global__ void __launch_bounds__(256) k_logits(const XT* __restrict__ x,
     }
 }
 
-// Large batches: a 128-token x 128-expert block tile, 8 x 8 (token, expert)
+// Large batches: a 64-token x 128-expert block tile, 4 x 8 (token, expert)
 // pairs per thread, 16 h per shared-memory stage with the next stage's
 // global loads held in registers while the current one is consumed.  The
 // arithmetic order is the same as k_logits: per 256-wide chunk a fused
 // multiply-add chain in ascending h, chunk sums added in ascending order.
-constexpr int kBigT = 128, kBigE = 128, kBigK = 16;
+constexpr int kBigT = 64, kBigE = 128, kBigK = 16;
 
 constexpr int kBigLd = kBigE + 4;  // row stride of the running sums in shared memory
 constexpr size_t kBigDynSmem = (size_t)kBigT * kBigLd * sizeof(float);
 
 template <typename XT>
-__global__ void __launch_bounds__(256, 1) k_logits_big(const XT* __restrict__ x,
+__global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
                                                        const float* __restrict__ wg, int T, int H,
                                                        int E, float* __restrict__ out) {
-    __shared__ __align__(16) float xs[2][kBigK][kBigT + 4];
+    __shared__ __align__(16) float xs[2][kBigK][kBigT + 4];  // [buffer][h][token]
     __shared__ __align__(16) float ws[2][kBigK][kBigE + 4];
     extern __shared__ float ls[];  // [kBigT][kBigLd]: sum of the finished chunks, per pair
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int e0 = blockIdx.x * kBigE, t0 = blockIdx.y * kBigT;
-    // loader mapping: x  -> token lt = tid / 2, h offset (tid % 2) * 8   (8 values)
-    //                 w  -> expert le = tid / 2, h offset (tid % 2) * 8   (8 values)
+    // loader mapping: w  -> expert lt = tid / 2, h offset (tid % 2) * 8   (8 values)
+    //                 x  -> token  lt (threads with lt < 64 only)
     const int lt = tid >> 1, lh = (tid & 1) * 8;
-    const bool xin = t0 + lt < T, win = e0 + lt < E;
+    const bool xload = lt < kBigT;
+    const bool xin = xload && t0 + lt < T, win = e0 + lt < E;
     const XT* xrow = x + (int64_t)(xin ? t0 + lt : 0) * H + lh;
     const float* wrow = wg + (int64_t)(win ? e0 + lt : 0) * H + lh;
     float rx[8], rw[8];
@@ -147,17 +203,18 @@ __global__ void __launch_bounds__(256, 1) k_logits_big(const XT* __restrict__ x,
     auto store = [&](int buf) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            xs[buf][lh + i][lt] = rx[i];
+            if (xload) xs[buf][lh + i][lt] = rx[i];
             ws[buf][lh + i][lt] = rw[i];
         }
     };
-    auto row_of = [&](int i) { return i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4; };
+    auto row_of = [&](int i) { return ty * 4 + i; };
     auto col_of = [&](int j) { return j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4; };
-    float p[8][8];
+    // p[i][q] holds the chain sums of columns col_of(2q), col_of(2q + 1)
+    uint64_t p[4][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) p[i][j] = 0.0f;
+        for (int q = 0; q < 4; ++q) p[i][q] = 0;
     const int nk = H / kBigK;
     load(0);
     store(0);
@@ -168,33 +225,38 @@ __global__ void __launch_bounds__(256, 1) k_logits_big(const XT* __restrict__ x,
 #pragma unroll
         for (int kk = 0; kk < kBigK; ++kk) {
             const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
-            const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][64 + ty * 4]);
             const float4 b0 = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * 4]);
             const float4 b1 = *reinterpret_cast<const float4*>(&ws[buf][kk][64 + tx * 4]);
-            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            const float a[4] = {a0.x, a0.y, a0.z, a0.w};
+            const uint64_t b[4] = {pack2(b0.x, b0.y), pack2(b0.z, b0.w), pack2(b1.x, b1.y),
+                                   pack2(b1.z, b1.w)};
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 4; ++i) {
+                const uint64_t ai = pack2(a[i], a[i]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) p[i][j] = __fmaf_rn(a[i], b[j], p[i][j]);
+                for (int q = 0; q < 4; ++q) fma2(p[i][q], ai, b[q]);
+            }
         }
         const int h_next = (kt + 1) * kBigK;
         if (h_next % kChunk == 0 || h_next >= H) {  // a 256-wide chunk ends here
             const bool first = (h_next - 1) / kChunk == 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float* l = &ls[row_of(i) * kBigLd + col_of(j)];
-                    *l = first ? p[i][j] : __fadd_rn(*l, p[i][j]);
-                    p[i][j] = 0.0f;
+                for (int q = 0; q < 4; ++q) {
+                    const float2 v = unpack2(p[i][q]);
+                    float* l0 = &ls[row_of(i) * kBigLd + col_of(2 * q)];
+                    float* l1 = &ls[row_of(i) * kBigLd + col_of(2 * q + 1)];
+                    *l0 = first ? v.x : __fadd_rn(*l0, v.x);
+                    *l1 = first ? v.y : __fadd_rn(*l1, v.y);
+                    p[i][q] = 0;
                 }
         }
         if (kt + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
         const int t = t0 + row_of(i);
         if (t >= T) continue;
 #pragma unroll
@@ -251,6 +313,26 @@ __device__ __forceinline__ void warp_best(float& k, int& i) {
     }
 }
 
+// Sum of the chunk partials of the split router, in chunk order:
+// l[t][e] = ((P_0 + P_1) + P_2) + ...  written over P_0.  One thread per
+// (token, expert); its loads are independent of each other.
+__global__ void __launch_bounds__(256) k_reduce_parts(float* __restrict__ parts, int nsplit,
+                                                      int64_t TE) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= TE) return;
+    float v[32];
+    const int n = nsplit < 32 ? nsplit : 32;
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+        if (c < n) v[c] = parts[(int64_t)c * TE + i];
+    float acc = v[0];
+#pragma unroll
+    for (int c = 1; c < 32; ++c)
+        if (c < n) acc = __fadd_rn(acc, v[c]);
+    for (int c = 32; c < nsplit; ++c) acc = __fadd_rn(acc, parts[(int64_t)c * TE + i]);
+    parts[i] = acc;
+}
+
 // One warp per token.  Lane `lane` holds experts e = lane + 32 v.
 template <int V>
 __global__ void __launch_bounds__(256) k_select(const float* __restrict__ logits, int nsplit, int T,
@@ -261,7 +343,7 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ logits
                                                 float* __restrict__ topk_w) {
     __shared__ float keys_sh[8][32 * V];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
     if (t >= T) return;
     const float kNegInf = -__int_as_float(0x7f800000);
     float lg[V], key[V], sc[V];
@@ -387,18 +469,18 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ logits
 }
 
 struct RoutePlan {
-    int tm;      // 2 or 4 (k_logits, TM == TN) or 8 (k_logits_big)
+    int tm;      // 2 or 4 (k_logits, TM == TN) or 8 (k_logits_big, 64 x 128 tiles)
     int nsplit;  // 1, or the number of 256-wide chunks
 };
 
 // Small batches split the h chunks over the grid (partial sums added in
-// order by k_select); large ones use the 128 x 128 tile when it fills the GPU.
+// order by k_select); large ones use the 64 x 128 tile when it fills the GPU.
 RoutePlan plan(const moe_route_cfg* c) {
     RoutePlan p;
     const int64_t tiles32 = (int64_t)((c->T + 31) / 32) * ((c->E + 31) / 32);
-    const int64_t tiles128 = (int64_t)((c->T + kBigT - 1) / kBigT) * ((c->E + kBigE - 1) / kBigE);
+    const int64_t tiles_big = (int64_t)((c->T + kBigT - 1) / kBigT) * ((c->E + kBigE - 1) / kBigE);
     const bool small = tiles32 < 512;
-    p.tm = small ? 2 : (tiles128 >= 120 ? 8 : 4);
+    p.tm = small ? 2 : (tiles_big >= 240 ? 8 : 4);
     p.nsplit = small ? (c->H + kChunk - 1) / kChunk : 1;
     return p;
 }
@@ -483,12 +565,22 @@ moe_status moe_route(const moe_route_cfg* c, const void* x, moe_dtype x_dtype, c
     else
         launch_logits(c, p, static_cast<const __nv_bfloat16*>(x), w_gate, lg, stream);
     SWB_LAUNCHED("moe_route: logits kernel");
-    const int blocks = (c->T + 7) / 8;
+    int nsplit = p.nsplit;
+    if (nsplit > 1) {   // chunk partials -> logits, in chunk order
+        const int64_t TE = (int64_t)c->T * c->E;
+        k_reduce_parts<<<(unsigned)((TE + 255) / 256), 256, 0, stream>>>(lg, nsplit, TE);
+        SWB_LAUNCHED("moe_route: partial-sum kernel");
+        nsplit = 1;
+    }
+    // one warp per token; small batches get one warp per block to use every SM
+    const int warps = c->T < 8 * 148 ? 1 : 8;
+    const int blocks = (c->T + warps - 1) / warps;
     const int V = (c->E + 31) / 32;
 #define SWB_SELECT(VV)                                                                        \
-    k_select<VV><<<blocks, 256, 0, stream>>>(lg, p.nsplit, c->T, c->E, c->k, c->score,        \
-                                             c->n_group, c->topk_group, c->routed_scale,      \
-                                             c->renormalize, bias, topk_idx, topk_w)
+    k_select<VV><<<blocks, 32 * warps, 0, stream>>>(lg, nsplit, c->T, c->E, c->k, c->score,   \
+                                                    c->n_group, c->topk_group,               \
+                                                    c->routed_scale, c->renormalize, bias,   \
+                                                    topk_idx, topk_w)
     if (V <= 1) SWB_SELECT(1);
     else if (V <= 2) SWB_SELECT(2);
     else if (V <= 4) SWB_SELECT(4);

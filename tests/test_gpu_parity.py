@@ -145,6 +145,23 @@ def test_empty_batch_is_a_no_op(cuda_device):
     assert dl.layer.offsets.cpu().numpy().tolist() == [0] * (cfg.E + 1)
 
 
+def test_kernel_launch_counter(cuda_device):
+    """moe_kernel_launches counts each accepted kernel launch: one layer of
+    300 tokens is the split router (chunk logits, partial sums, selection),
+    permute (histogram, scan, scatter, gather), the two grouped GEMM kernels
+    and the combine; a 0-token layer launches nothing."""
+    dl = mdev.build_layer(MID_SIGMOID)
+    sync_check()
+    n0 = L.moe_kernel_launches()
+    dl.layer.forward(dl.x)
+    assert L.moe_kernel_launches() - n0 == 3 + 4 + 2 + 1
+    empty = mdev.build_layer(MID_SIGMOID.with_(cfg_id=16, T=0))
+    n0 = L.moe_kernel_launches()
+    empty.layer.forward(empty.x)
+    assert L.moe_kernel_launches() == n0
+    sync_check()
+
+
 def test_out_of_range_expert_index_is_reported(cuda_device):
     cfg = SPARSE_DECODE
     dl = mdev.build_layer(cfg)
