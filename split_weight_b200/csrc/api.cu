@@ -46,6 +46,8 @@ bool cuda_injected_failure() {
 }
 
 moe_status cuda_check(cudaError_t e, const char* what) {
+    // reported here: clear it so the next launch check does not report it again
+    (void)cudaGetLastError();
     return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 

@@ -23,12 +23,13 @@ struct CfgF8 {
     static constexpr uint32_t kPartCols = kNA * BN;                 // one partial-sum set
     static constexpr int kPBufs = (512 / kPartCols) >= 8 ? 8 : (512 / kPartCols);
     static constexpr uint32_t kTmemCols = kPBufs * kPartCols;
-    static constexpr int kEpiWarps = 8;                             // 2 per TMEM lane quarter
+    static constexpr int kEpiWarps = BN >= 64 ? 16 : 8;             // 4 or 2 per TMEM lane quarter
+    static constexpr int kParts = kEpiWarps / 4;                    // column slices of the tile
     static constexpr int kThreads = 64 + 32 * kEpiWarps;
     static constexpr int kRowsPerTile = MODE == kPair ? 2 * kBM : kBM;
-    static constexpr int kCols = BN / 2;                            // columns per epilogue warp
-    // per-warp combined scales [8][2][kCols] + amax exchange [2 halves][2 tiles][4][kCols]
-    static constexpr size_t kScratch = (size_t)kEpiWarps * 2 * kCols * 4 + 2 * 2 * 4 * kCols * 4;
+    static constexpr int kCols = BN / kParts;                       // columns per epilogue warp
+    // per-warp combined scales [kEpiWarps][2][kCols] + amax exchange [kParts][2 tiles][4][kCols]
+    static constexpr size_t kScratch = (size_t)kEpiWarps * 2 * kCols * 4 + (size_t)kParts * 2 * 4 * kCols * 4;
     static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024 + kScratch;
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                   "TMEM allocation must be a power of two in [32, 512]");
@@ -50,7 +51,7 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
     extern __shared__ uint8_t dyn_smem[];
     __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
     __shared__ __align__(8) uint64_t part_full[C::kPBufs], part_empty[C::kPBufs];
-    __shared__ __align__(8) uint64_t half_bar[2];   // the 4 epilogue warps of one column half
+    __shared__ __align__(8) uint64_t half_bar[C::kParts];  // the 4 epilogue warps of one column slice
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ Tables tb;
@@ -75,8 +76,7 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
             mbar_init(smem_u32(&part_full[b]), 1);
             mbar_init(smem_u32(&part_empty[b]), C::kEpiWarps);
         }
-        mbar_init(smem_u32(&half_bar[0]), 4);
-        mbar_init(smem_u32(&half_bar[1]), 4);
+        for (int b = 0; b < C::kParts; ++b) mbar_init(smem_u32(&half_bar[b]), 4);
         fence_mbar_init();
         tma_prefetch_map(&p.act_map);
         tma_prefetch_map(&p.act_map64);
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
         // ------------------------------------------------ epilogue (warps 2..9)
         constexpr int kC = C::kCols;
         const int q = warp & 3;              // TMEM lane quarter this warp may access
-        const int part = (warp - 2) >> 2;    // which half of the token columns
+        const int part = (warp - 2) >> 2;    // which slice of the token columns
         const int e = warp - 2;
         const int c_begin = part * kC;
         float* cg = scratch + e * 2 * kC;    // this warp's combined scales, gate / row block 0
