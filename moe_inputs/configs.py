@@ -105,6 +105,8 @@ CONFIGS: dict[int, MoEConfig] = {
 # the 128-token decode step), the prefill shape and the FP8 shape with 32 experts.
 PROFILE_CASES: dict[int, MoEConfig] = {
     21: CONFIGS[2].with_(cfg_id=21, name="r1_decode_shape_E32_T16", T=16, E=32, local_count=8),
+    # the 8K-prefill router (T, H, E as in the prefill workload) with small experts
+    22: CONFIGS[3].with_(cfg_id=22, name="r1_router_shape_T8192_I128", I=128),
     23: CONFIGS[3].with_(cfg_id=23, name="r1_prefill_shape_E32_T1024", T=1024, E=32,
                          local_count=8),
     25: CONFIGS[5].with_(cfg_id=25, name="r1_fp8_shape_E32_T512", T=512, E=32, local_count=8,
