@@ -74,3 +74,24 @@ def test_roofline_figures_decode_shape():
 def test_default_arguments():
     a = bench.parse_args([])
     assert (a.gpus, a.config, a.impl) == (1, 2, "ours") and a.warmup >= 3
+
+
+def test_profiled_traffic_scaling_and_staleness(tmp_path, monkeypatch):
+    """A full-size workload's traffic is its reduced case's measured bytes scaled
+    by the ratio of algorithmic bytes; a changed kernel source voids it."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "split_weight_b200" / "csrc").mkdir(parents=True)
+    (tmp_path / "split_weight_b200" / "csrc" / "k.cuh").write_text("kernel v1")
+    h = bench.kernel_source_hash(["k.cuh"])
+    rec = {"small": {"kernel_files": ["k.cuh"], "kernel_source_hash": h,
+                     "dram_bytes_per_call": 1100, "algorithmic_bytes_per_call": 1000},
+           "full": {"scaled_from": "small"}}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(path))
+    assert bench.profiled_traffic("small", 1000.0) == 1100
+    assert bench.profiled_traffic("full", 5000.0) == 5500
+    assert bench.profiled_traffic("absent", 5000.0) is None
+    (tmp_path / "split_weight_b200" / "csrc" / "k.cuh").write_text("kernel v2")
+    assert bench.profiled_traffic("full", 5000.0) is None
