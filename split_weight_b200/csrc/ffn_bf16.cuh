@@ -23,7 +23,8 @@ struct Cfg {
     static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
     static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
     static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
-    static constexpr int kEpiWarps = BN >= 256 ? 8 : 4;
+    // one TMEM buffer at BN=256: its epilogue stalls the MMA, so it gets 16 warps
+    static constexpr int kEpiWarps = BN >= 256 ? (W8 ? 8 : 16) : 4;
     static constexpr int kConvWarps = W8 ? kConvThreads / 32 : 0;
     static constexpr int kConvFirstWarp = 2 + kEpiWarps;
     static constexpr int kThreads = 64 + 32 * (kEpiWarps + kConvWarps);
@@ -240,8 +241,8 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     } else {
         // ------------------------------------------------ epilogue
         const int q = warp & 3;                    // TMEM lane quarter this warp may access
-        const int part = (warp - 2) >> 2;          // column half (8 epilogue warps) or 0
-        constexpr int kCols = C::kEpiWarps == 8 ? BN / 2 : BN;
+        const int part = (warp - 2) >> 2;          // column slice of this warp's lane quarter
+        constexpr int kCols = BN / (C::kEpiWarps / 4);
         int acc = 0;
         uint32_t acc_use[2] = {0u, 0u};
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
