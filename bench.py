@@ -48,6 +48,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-merge-ablation", action="store_true")
+    p.add_argument("--prefetch-split", type=int, default=1, choices=(0, 1),
+                   help="issue each layer's fetch in two halves in the windows between grouped GEMMs")
     return p.parse_args(argv)
 
 
@@ -210,7 +212,8 @@ def run_ours(args, rank, world, local_rank):
         from split_weight_b200 import PrefetchPipeline
         stores = [mdev.peer_store(cfg, l, dls[l].layer.weights, dev) for l in range(cfg.layers)]
         rbytes = dls[0].layer.weights.n_remote * dls[0].layer.weights.stride
-        pipe = PrefetchPipeline([d.layer for d in dls], stores, rbytes, dev)
+        pipe = PrefetchPipeline([d.layer for d in dls], stores, rbytes, dev,
+                                split=args.prefetch_split)
         for d in dls:  # the layers' own remote pools are not needed: the buffers replace them
             d.layer.weights.remote = torch.empty(1, dtype=torch.uint8, device=dev)
         torch.cuda.empty_cache()
@@ -295,6 +298,7 @@ def run_ours(args, rank, world, local_rank):
         piped_ms = elapsed_ms / args.steps
         exposed = max(0.0, (piped_ms - nocopy_ms) / cfg.layers)
         prefetch_info = {
+            "schedule": "halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM",
             "remote_bytes_per_layer": pipe.remote_bytes,
             "copy_alone_ms_per_layer": round(copy_ms, 4),
             "step_ms_pipelined": round(piped_ms, 4),

@@ -212,12 +212,20 @@ class PrefetchPipeline:
     GEMM.  With wrap=True the fetches issued by the last layers of a pass are
     those of the next pass's first layers, as in a steady stream of forward
     passes.
+
+    With split=True each fetch is issued in two halves: the first after
+    execution g's grouped GEMMs, the second after execution g + 1's, and
+    ready is recorded after the second.  Each half then starts in the window
+    of routing, permutation and combine between two grouped GEMMs instead of
+    the whole fetch running beside the next grouped GEMM.
     """
 
     def __init__(self, layers: list[MoELayer], peer_stores: list[torch.Tensor],
-                 remote_bytes: int, device: torch.device | str = "cuda", chunk_bytes: int = 0):
+                 remote_bytes: int, device: torch.device | str = "cuda", chunk_bytes: int = 0,
+                 split: bool = True):
         self.layers, self.peer_stores = layers, peer_stores
         self.remote_bytes, self.chunk_bytes = remote_bytes, chunk_bytes
+        self.split, self.pending = split, None
         dev = torch.device(device)
         self.bufs = [torch.empty(max(remote_bytes, 1), dtype=torch.uint8, device=dev)
                      for _ in range(2)]
@@ -236,9 +244,20 @@ class PrefetchPipeline:
                                      wait_free.cuda_event if wait_free is not None else None,
                                      self.ready[buf].cuda_event))
 
+    def fetch_half(self, layer: int, buf: int, half: int, wait_free: torch.cuda.Event) -> None:
+        """One half of a fetch; the second half records ready[buf]."""
+        cut = (self.remote_bytes // 2) // 256 * 256
+        lo, hi = (0, cut) if half == 0 else (cut, self.remote_bytes)
+        assert wait_free.cuda_event != 0 and self.ready[buf].cuda_event != 0
+        L.check(L.moe_prefetch_layer(self.peer_stores[layer].data_ptr() + lo,
+                                     self.bufs[buf].data_ptr() + lo, hi - lo, self.chunk_bytes,
+                                     self.copy_stream.cuda_stream, wait_free.cuda_event,
+                                     self.ready[buf].cuda_event if half == 1 else None))
+
     def prime(self) -> None:
         """Enqueues the fetches of the next two executions (before a run)."""
         n = len(self.layers)
+        self.pending = None
         for i in range(2):
             self.prefetch((self.g + i) % n, (self.g + i) % 2, None)
 
@@ -257,7 +276,15 @@ class PrefetchPipeline:
         layer.grouped_ffn(h, self.bufs[b])
         if ffn_events is not None:
             ffn_events[1].record(stream)
-        if prefetch and (l + 2 < n or wrap):
+        if prefetch and self.split:
+            self.free[b].record(stream)
+            if self.pending is not None:  # second half of execution g + 1's fetch
+                self.fetch_half(*self.pending, 1, self.free[b])
+                self.pending = None
+            if l + 2 < n or wrap:        # first half of execution g + 2's
+                self.fetch_half((l + 2) % n, b, 0, self.free[b])
+                self.pending = ((l + 2) % n, b)
+        elif prefetch and (l + 2 < n or wrap):
             self.free[b].record(stream)
             self.prefetch((l + 2) % n, b, self.free[b])
         layer.combine(h)

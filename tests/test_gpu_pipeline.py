@@ -20,7 +20,8 @@ def _free_memory(cuda_device):
     torch.cuda.empty_cache()
 
 
-def test_pipeline_equals_resident_layers():
+@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
+def test_pipeline_equals_resident_layers(split):
     """Three layers through two alternate buffers, each filled by
     moe_prefetch_layer from the layer's peer store, give the same bits as
     each layer computed with its own resident remote pool."""
@@ -36,7 +37,7 @@ def test_pipeline_equals_resident_layers():
         assert torch.equal(stores[l], dls[l].layer.weights.remote)
     w0 = dls[0].layer.weights
     pipe = PrefetchPipeline([d.layer for d in dls], stores, w0.n_remote * w0.stride,
-                            chunk_bytes=1 << 20)
+                            chunk_bytes=1 << 20, split=split)
     for d in dls:
         d.layer.weights.remote.zero_()   # the pipeline must not read them
     with torch.cuda.stream(pipe.copy_stream):
