@@ -11,7 +11,7 @@
 // One persistent, warp-specialised kernel per GEMM (sm_100a):
 //   warp 0      TMA producer (one thread): weight tile(s) + token rows
 //   warp 1      tcgen05.mma issuer (one thread); owns the TMEM allocation
-//   warps 2..   epilogue (4 or 8 warps): TMEM -> registers -> (SwiGLU) -> bf16
+//   warps 2..   epilogue (4, 8 or 16 warps): TMEM -> registers -> (SwiGLU) -> bf16
 // The MMA puts weight rows on M (128 per instruction) and the expert's tokens
 // on N (16..256), so a decode-sized expert with 4 tokens costs an N=16 MMA,
 // not a 128-row tile.  A CTA holds one or two weight tiles per stage:
@@ -23,7 +23,8 @@
 // each MMA needs.  Accumulators are double buffered in TMEM when they fit
 // (two buffers of up to 256 columns) so the epilogue of one tile overlaps
 // the next tile's main loop; the widest tiles (2 x 256 columns) use all 512
-// TMEM columns in one buffer and 8 epilogue warps.
+// TMEM columns in one buffer and 16 epilogue warps, so the epilogue that
+// holds up the next tile's MMA is short.
 #include "ffn_bf16.cuh"
 #include "ffn_f8.cuh"
 
