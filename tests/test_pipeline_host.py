@@ -1,0 +1,170 @@
+"""The prefetch schedule of PrefetchPipeline on the host (no GPU work).
+
+Streams, events and the copy call are replaced by fakes that log, in host
+order, what each stream is asked to do.  A small replay then runs the two
+streams with CUDA's event rule (a wait is for the last record of the event
+enqueued before it) and checks that every grouped GEMM reads a buffer fully
+refilled with its own layer's remote experts, for both fetch schedules."""
+import pytest
+import torch
+
+import split_weight_b200.layer as layer_mod
+from split_weight_b200 import _lib as L
+
+
+class Log:
+    ops: list = []
+
+
+class FakeEvent:
+    count = 0
+    by_id: dict = {}
+
+    def __init__(self):
+        FakeEvent.count += 1
+        self.cuda_event = FakeEvent.count
+        self.version = 0  # records enqueued so far (host order)
+        FakeEvent.by_id[self.cuda_event] = self
+
+    def record(self, stream=None):
+        self.version += 1
+        Log.ops.append(("record", getattr(stream, "name", "compute"), self, self.version))
+
+
+class FakeStream:
+    def __init__(self, device=None, name="copy"):
+        self.name = name
+        self.cuda_stream = name
+
+    def wait_event(self, ev):
+        Log.ops.append(("wait", self.name, ev, ev.version))
+
+
+class Ptr(tuple):
+    """A device pointer stand-in: (owner, byte offset)."""
+
+    def __add__(self, k):
+        return Ptr((self[0], self[1] + k))
+
+
+class Buffer:
+    def __init__(self, owner):
+        self.owner = owner
+
+    def data_ptr(self):
+        return Ptr((self.owner, 0))
+
+
+class FakeLayer:
+    def __init__(self, idx):
+        self.idx, self.y = idx, None
+
+    def route(self, x, h):
+        pass
+
+    def permute(self, x, h):
+        pass
+
+    def grouped_ffn(self, h, remote):
+        Log.ops.append(("ffn", "compute", self.idx, remote.owner))
+
+    def combine(self, h):
+        pass
+
+
+def fake_prefetch(src, dst, nbytes, chunk, stream, wait, ready):
+    if wait is not None:
+        ev = FakeEvent.by_id[wait]
+        Log.ops.append(("wait", "copy", ev, ev.version))
+    assert src[1] == dst[1]
+    Log.ops.append(("copy", "copy", src[0], dst[0], src[1], src[1] + nbytes))
+    if ready is not None:
+        FakeEvent.by_id[ready].record(FakeStream(name="copy"))
+    return L.MOE_OK
+
+
+def replay(ops, nbytes):
+    """Runs both streams in order, honouring waits; returns (layer, buffer
+    contents) for every grouped GEMM in execution order."""
+    done = {}  # event id -> highest executed record version
+    queues = {s: [o for o in ops if o[1] == s] for s in ("compute", "copy")}
+    pos = {s: 0 for s in queues}
+    buffers, seen, moved = {}, [], True
+    while moved:
+        moved = False
+        for s, q in queues.items():
+            while pos[s] < len(q):
+                op = q[pos[s]]
+                if op[0] == "wait" and done.get(op[2].cuda_event, 0) < op[3]:
+                    break
+                if op[0] == "record":
+                    done[op[2].cuda_event] = max(done.get(op[2].cuda_event, 0), op[3])
+                elif op[0] == "copy":
+                    _, _, layer, buf, lo, hi = op
+                    content = buffers.setdefault(buf, [None] * nbytes)
+                    content[lo:hi] = [layer] * (hi - lo)
+                elif op[0] == "ffn":
+                    seen.append((op[2], list(buffers.get(op[3], [None] * nbytes))))
+                pos[s] += 1
+                moved = True
+    assert all(pos[s] == len(q) for s, q in queues.items()), "the schedule deadlocks"
+    return seen
+
+
+@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
+@pytest.mark.parametrize("n_layers", [1, 2, 3, 4])
+def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_layers):
+    monkeypatch.setattr(torch.cuda, "Stream", FakeStream)
+    monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
+    monkeypatch.setattr(L, "moe_prefetch_layer", fake_prefetch)
+    monkeypatch.setattr(L, "check", lambda status: None)
+    Log.ops = []
+    nbytes = 1000  # an odd size: the halves split at a 256-byte boundary
+
+    # the constructor's device allocations replaced by pointer stand-ins
+    pipe = layer_mod.PrefetchPipeline.__new__(layer_mod.PrefetchPipeline)
+    pipe.layers = [FakeLayer(l) for l in range(n_layers)]
+    pipe.peer_stores = [Buffer(("store", l)) for l in range(n_layers)]
+    pipe.remote_bytes, pipe.chunk_bytes = nbytes, 0
+    pipe.split, pipe.pending = split, None
+    pipe.bufs = [Buffer(("buf", 0)), Buffer(("buf", 1))]
+    pipe.copy_stream = FakeStream(name="copy")
+    pipe.ready = [FakeEvent() for _ in range(2)]
+    pipe.free = [FakeEvent() for _ in range(2)]
+    for ev in pipe.ready + pipe.free:
+        ev.record(pipe.copy_stream)
+    pipe.g = 0
+
+    compute = FakeStream(name="compute")
+    pipe.prime()
+    n_exec = 3 * n_layers + 1
+    for i in range(n_exec):
+        pipe.run_layer(i % n_layers, None, compute, prefetch=True, wrap=True)
+
+    seen = replay(Log.ops, nbytes)
+    assert len(seen) == n_exec
+    for i, (lidx, content) in enumerate(seen):
+        assert lidx == i % n_layers
+        assert all(c == ("store", lidx) for c in content), (
+            f"execution {i} (layer {lidx}) read {sorted(set(map(str, content)))}")
+
+
+def test_split_halves_cover_the_buffer_once(monkeypatch):
+    """fetch_half(0) and fetch_half(1) copy [0, cut) and [cut, n) with cut a
+    256-byte multiple; only the second records ready."""
+    calls = []
+    monkeypatch.setattr(L, "moe_prefetch_layer",
+                        lambda s, d, n, c, st, w, r: calls.append((s[1], n, r)) or L.MOE_OK)
+    monkeypatch.setattr(L, "check", lambda status: None)
+    pipe = layer_mod.PrefetchPipeline.__new__(layer_mod.PrefetchPipeline)
+    pipe.peer_stores = [Buffer("store")]
+    pipe.bufs = [Buffer("buf0"), Buffer("buf1")]
+    pipe.remote_bytes, pipe.chunk_bytes = 16_911_433_728, 0
+    pipe.copy_stream = FakeStream(name="copy")
+    pipe.ready = [FakeEvent(), FakeEvent()]
+    free = FakeEvent()
+    pipe.fetch_half(0, 1, 0, free)
+    pipe.fetch_half(0, 1, 1, free)
+    (lo0, n0, r0), (lo1, n1, r1) = calls
+    assert lo0 == 0 and lo1 == n0 and n0 + n1 == pipe.remote_bytes and n0 % 256 == 0
+    assert r0 is None and r1 == pipe.ready[1].cuda_event
