@@ -474,7 +474,8 @@ struct RoutePlan {
 };
 
 // Small batches split the h chunks over the grid (partial sums added in
-// order by k_select); large ones use the 64 x 128 tile when it fills the GPU.
+// chunk order by k_reduce_parts); large ones use the 64 x 128 tile when it
+// fills the GPU.
 RoutePlan plan(const moe_route_cfg* c) {
     RoutePlan p;
     const int64_t tiles32 = (int64_t)((c->T + 31) / 32) * ((c->E + 31) / 32);
