@@ -95,3 +95,25 @@ def test_profiled_traffic_scaling_and_staleness(tmp_path, monkeypatch):
     assert bench.profiled_traffic("absent", 5000.0) is None
     (tmp_path / "split_weight_b200" / "csrc" / "k.cuh").write_text("kernel v2")
     assert bench.profiled_traffic("full", 5000.0) is None
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` runs the CPU oracle and prints exactly one JSON
+    line with the contract's keys (run as a subprocess, as the driver does)."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "1"], cwd=root, capture_output=True,
+                         text=True, timeout=600, check=True).stdout
+    lines = [l for l in out.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "impl",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
