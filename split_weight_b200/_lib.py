@@ -53,7 +53,7 @@ class MoEError(RuntimeError):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: run split_weight_b200.build.build() "
+    raise ImportError(f"{LIB_PATH} is missing: run python split_weight_b200/build.py "
                       "(the CUDA library is required; there is no CPU fallback)")
 _lib = ctypes.CDLL(LIB_PATH)
 
