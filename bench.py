@@ -50,6 +50,14 @@ def parse_args(argv=None):
     p.add_argument("--no-merge-ablation", action="store_true")
     p.add_argument("--prefetch-split", type=int, default=1, choices=(0, 1),
                    help="issue each layer's fetch in two halves in the windows between grouped GEMMs")
+    p.add_argument("--act-dtype", choices=["bf16", "e4m3"], default="bf16",
+                   help="activations the grouped GEMMs read (e4m3: opt-in fp8 tensor-core path, "
+                        "e4m3-weight workloads only)")
+    p.add_argument("--workloads", default="3,5",
+                   help="further workloads measured in the same run (1 GPU only; '' for none)")
+    p.add_argument("--workload-steps", type=int, default=5)
+    p.add_argument("--measure-peaks", action="store_true",
+                   help="measure the fp8 dense GEMM peak and the read-only HBM peak, print JSON")
     return p.parse_args(argv)
 
 
@@ -62,6 +70,39 @@ def load_peaks():
         return d, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+EXTRA_PEAKS = os.path.join(ROOT, "profiles", "peaks_fp8_hbm_read.json")
+SUSTAINED_AFTER_S = 2.0   # timed regions at least this long are compared with the sustained peak
+
+
+def load_extra_peaks():
+    """fp8 dense TFLOP/s and read-only HBM GB/s measured by `bench.py
+    --measure-peaks` on this machine's B200s (committed under profiles/)."""
+    try:
+        with open(EXTRA_PEAKS) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return {}
+
+
+def tensor_peak(peaks, mma_kind: str, timed_s: float):
+    """(peak TFLOP/s, its source) for the MMA kind the kernel issues: the burst
+    figure for a timed region shorter than SUSTAINED_AFTER_S, else the
+    sustained one.  kind::f16 takes the bf16 figures; kind::f8f6f4 the
+    measured fp8 figure, else bf16 x 2 (the nominal ratio)."""
+    sustained = timed_s >= SUSTAINED_AFTER_S and "bf16_tflops_sustained" in peaks
+    bf16 = float(peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
+    which = "sustained" if sustained else "burst"
+    if mma_kind == "f16":
+        return bf16, f"bf16 dense, {which}"
+    extra = load_extra_peaks()
+    if "fp8_tflops" in extra:
+        fp8 = float(extra["fp8_tflops"])
+        if sustained:   # scale the measured burst figure like the bf16 one
+            fp8 *= float(peaks["bf16_tflops_sustained"]) / float(peaks["bf16_tflops"])
+        return fp8, f"fp8 dense measured (torch._scaled_mm 8192^3), {which}"
+    return 2.0 * bf16, f"fp8 dense taken as 2 x bf16 {which} (nominal ratio)"
 
 
 def kernel_source_hash(files) -> str:
@@ -195,18 +236,13 @@ def roofline_figures(cfg, counts_per_layer, peaks):
 
 
 # ----------------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
+def build_workload(cfg, args, dev, act_dtype):
+    """Every layer of the workload resident in HBM; for multi-layer workloads
+    the remote experts only in their peer stores, fetched by the pipeline."""
     import torch
-    from moe_inputs import config, device as mdev
-
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    cfg = config(args.config)
-    stream = torch.cuda.Stream(device=dev)
-    torch.cuda.set_stream(stream)
-
-    # ---- workload (resident in HBM before timing)
-    dls = [mdev.build_layer(cfg, layer=l, device=dev) for l in range(cfg.layers)]
+    from moe_inputs import device as mdev
+    dls = [mdev.build_layer(cfg, layer=l, device=dev, act_dtype=act_dtype)
+           for l in range(cfg.layers)]
     pipe = None
     if cfg.layers > 1:
         from split_weight_b200 import PrefetchPipeline
@@ -219,7 +255,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         pipe.prime()
     torch.cuda.synchronize()
+    return dls, pipe
 
+
+def make_step(cfg, dls, pipe, stream):
     xs = [d.x for d in dls]
     h = stream.cuda_stream
 
@@ -239,6 +278,166 @@ def run_ours(args, rank, world, local_rank):
         for l in range(cfg.layers):
             pipe.run_layer(l, inputs[l], stream, prefetch=prefetch,
                            ffn_events=None if timed_ffn is None else timed_ffn[l])
+    return step
+
+
+def roofline_object(cfg, counts, act_dtype, ffn_ms, timed_s, peaks, peak_src):
+    """The `roofline` object of the grouped FFN call (its two launches)."""
+    flops, nbytes = roofline_figures(cfg, counts, peaks)
+    hbm = float(peaks["hbm_gbs"])
+    mma_kind = "f8f6f4" if act_dtype == "e4m3" else "f16"
+    tc_peak, tc_src = tensor_peak(peaks, mma_kind, timed_s)
+    t_hbm = nbytes / (hbm * 1e9)
+    t_flop = flops / (tc_peak * 1e12)
+    ffn_s = ffn_ms / 1e3
+    if t_hbm >= t_flop:
+        achieved = nbytes / ffn_s / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4)}
+        read_peak = load_extra_peaks().get("hbm_read_gbs")
+        if read_peak:
+            roof["frac_of_read_peak"] = round(achieved / float(read_peak), 4)
+            roof["read_peak_gbs"] = float(read_peak)
+    else:
+        achieved = flops / ffn_s / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(tc_peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4)}
+        if mma_kind == "f16" and "bf16_tflops_sustained" in peaks:
+            roof["frac_of_sustained"] = round(achieved / float(peaks["bf16_tflops_sustained"]), 4)
+            roof["frac_of_burst"] = round(achieved / float(peaks["bf16_tflops"]), 4)
+    traffic = profiled_traffic(cfg.name + ("" if act_dtype == "bf16" else "_" + act_dtype),
+                               nbytes / cfg.layers)
+    roof.update({
+        "traffic": (round(traffic * cfg.layers) if traffic is not None else None),
+        "kernel": "moe_grouped_ffn (gate/up + down launches)",
+        "mma_kind": mma_kind,
+        "peak_source": (f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+                        + (f"; tensor: {tc_src}" if roof["bound"] == "tensor" else "")),
+        "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+        "kernel_ms_per_step": round(ffn_ms, 4),
+        "roof_ms_per_step": round(max(t_hbm, t_flop) * 1e3, 4),
+        "frac_of_roof": round(max(t_hbm, t_flop) / ffn_s, 4),
+    })
+    return roof
+
+
+def time_steps(step, cfg, steps, stream, barrier, local_rank, sample_clocks=True):
+    """Times `steps` steps on the compute stream; the grouped FFN of every
+    layer is bracketed by its own events.  Returns (elapsed ms, FFN ms per
+    step, launches, clocks summary)."""
+    import torch
+    from split_weight_b200 import _lib as L
+
+    def events(n):
+        return [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(cfg.layers)] for _ in range(n)]
+    ffn_ev = events(steps)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local_rank) if sample_clocks else None
+    if clk is not None:
+        clk.__enter__()
+    try:
+        launches0 = L.moe_kernel_launches()
+        ev0.record(stream)
+        for i in range(steps):
+            step(ffn_ev[i])
+        ev1.record(stream)
+        launches = L.moe_kernel_launches() - launches0
+        torch.cuda.synchronize()
+    finally:
+        if clk is not None:
+            clk.__exit__(None, None, None)
+    elapsed_ms = ev0.elapsed_time(ev1)
+    ffn_ms = sum(a.elapsed_time(b) for st in ffn_ev for a, b in st) / steps
+    return elapsed_ms, ffn_ms, launches, (clk.summary() if clk is not None else None)
+
+
+def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
+    """Exposed copy time per layer: the same steps without copies, and the
+    copy of one layer's remote experts alone."""
+    import torch
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(3, min(steps, 10))
+    e0.record(stream)
+    for _ in range(reps):
+        step(prefetch=False)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    nocopy_ms = e0.elapsed_time(e1) / reps
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(pipe.copy_stream)
+    pipe.prefetch(0, 0, None)
+    c1.record(pipe.copy_stream)
+    torch.cuda.synchronize()
+    copy_ms = c0.elapsed_time(c1)
+    pipe.g = 0
+    pipe.prime()
+    torch.cuda.synchronize()
+    exposed = max(0.0, (piped_ms - nocopy_ms) / cfg.layers)
+    return {
+        "schedule": "halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM",
+        "remote_bytes_per_layer": pipe.remote_bytes,
+        "copy_alone_ms_per_layer": round(copy_ms, 4),
+        "step_ms_pipelined": round(piped_ms, 4),
+        "step_ms_no_copy": round(nocopy_ms, 4),
+        "exposed_copy_ms_per_layer": round(exposed, 4),
+        "hidden_fraction": round(1.0 - exposed / copy_ms, 4) if copy_ms > 0 else None,
+    }
+
+
+def measure_extra_workload(cfg_id, args, dev, stream, peaks, peak_src):
+    """Tokens/s, roofline and (multi-layer) prefetch overlap of another
+    workload, measured in the same run with a few steps."""
+    import gc
+    import torch
+    from moe_inputs import config
+    from split_weight_b200 import _lib as L
+    cfg = config(cfg_id)
+    act = args.act_dtype if cfg.w_dtype == "e4m3" else "bf16"
+    dls, pipe = build_workload(cfg, args, dev, act)
+    step = make_step(cfg, dls, pipe, stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    L.check(L.moe_check_device())
+    counts = [np.diff(d.layer.offsets.cpu().numpy()) for d in dls]
+    elapsed_ms, ffn_ms, launches, clocks = time_steps(step, cfg, args.workload_steps, stream,
+                                                      lambda: None, 0)
+    L.check(L.moe_check_device())
+    out = {"workload": workload_desc(cfg), "act_dtype": act, "steps": args.workload_steps,
+           "ms_per_step": round(elapsed_ms / args.workload_steps, 4),
+           "value": round(cfg.T * cfg.layers * args.workload_steps / (elapsed_ms / 1e3), 3),
+           "unit": "tokens/s", "gpu_launches": int(launches),
+           "roofline": roofline_object(cfg, counts, act, ffn_ms, elapsed_ms / 1e3, peaks, peak_src),
+           "clocks": clocks}
+    if pipe is not None:
+        out["prefetch"] = prefetch_overlap(cfg, pipe, step, stream,
+                                           elapsed_ms / args.workload_steps, args.workload_steps)
+    del dls, pipe, step
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from moe_inputs import config
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = config(args.config)
+    act_dtype = args.act_dtype if cfg.w_dtype == "e4m3" else "bf16"
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+
+    # ---- workload (resident in HBM before timing)
+    dls, pipe = build_workload(cfg, args, dev, act_dtype)
+    xs = [d.x for d in dls]
+    step = make_step(cfg, dls, pipe, stream)
 
     def barrier():
         if world > 1:
@@ -253,59 +452,16 @@ def run_ours(args, rank, world, local_rank):
     counts = [np.diff(d.layer.offsets.cpu().numpy()) for d in dls]
 
     # ---- device-timed region (FFN launches bracketed by their own events)
-    def events(n):
-        return [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(cfg.layers)] for _ in range(n)]
-    ffn_ev = events(args.steps)
-    barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
-        launches0 = L.moe_kernel_launches()
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(ffn_ev[i])
-        ev1.record(stream)
-        launches = L.moe_kernel_launches() - launches0
-        torch.cuda.synchronize()
-    elapsed_ms = ev0.elapsed_time(ev1)
-    ffn_ms = sum(a.elapsed_time(b) for st in ffn_ev for a, b in st) / args.steps
+    elapsed_ms, ffn_ms, launches, clocks = time_steps(step, cfg, args.steps, stream, barrier,
+                                                      local_rank)
     barrier()
     L.check(L.moe_check_device())
 
     # ---- pipelined workloads: exposed copy time per layer
     prefetch_info = None
     if pipe is not None:
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = max(3, min(args.steps, 10))
-        e0.record(stream)
-        for _ in range(reps):
-            step(prefetch=False)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        nocopy_ms = e0.elapsed_time(e1) / reps
-        # copy alone
-        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        c0.record(pipe.copy_stream)
-        pipe.prefetch(0, 0, None)
-        c1.record(pipe.copy_stream)
-        torch.cuda.synchronize()
-        copy_ms = c0.elapsed_time(c1)
-        pipe.g = 0
-        pipe.prime()
-        torch.cuda.synchronize()
-        piped_ms = elapsed_ms / args.steps
-        exposed = max(0.0, (piped_ms - nocopy_ms) / cfg.layers)
-        prefetch_info = {
-            "schedule": "halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM",
-            "remote_bytes_per_layer": pipe.remote_bytes,
-            "copy_alone_ms_per_layer": round(copy_ms, 4),
-            "step_ms_pipelined": round(piped_ms, 4),
-            "step_ms_no_copy": round(nocopy_ms, 4),
-            "exposed_copy_ms_per_layer": round(exposed, 4),
-            "hidden_fraction": round(1.0 - exposed / copy_ms, 4) if copy_ms > 0 else None,
-        }
+        prefetch_info = prefetch_overlap(cfg, pipe, step, stream, elapsed_ms / args.steps,
+                                         args.steps)
 
     # ---- split-weight ablation: merge both pools into one buffer every step
     merge_info = None
@@ -384,35 +540,9 @@ def run_ours(args, rank, world, local_rank):
         e2e["value"] = round(total_tokens / (e2e.pop("_ms") / 1e3), 3)
 
     peaks, peak_src = load_peaks()
-    flops, nbytes = roofline_figures(cfg, counts, peaks)
-    hbm = float(peaks["hbm_gbs"])
-    tc_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    if cfg.w_dtype == "e4m3":
-        tc_peak *= 2.0  # fp8 dense = 2x bf16 (nominal ratio)
-    t_hbm = nbytes / (hbm * 1e9)
-    t_flop = flops / (tc_peak * 1e12)
-    ffn_s = ffn_ms / 1e3
+    roof = roofline_object(cfg, counts, act_dtype, ffn_ms, elapsed_ms / 1e3, peaks, peak_src)
     workload = cfg.name
-    if t_hbm >= t_flop:
-        achieved = nbytes / ffn_s / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4)}
-    else:
-        achieved = flops / ffn_s / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4)}
-    traffic = profiled_traffic(workload, nbytes / cfg.layers)
-    roof.update({
-        "traffic": (round(traffic * cfg.layers) if traffic is not None else None),
-        "kernel": "moe_grouped_ffn (gate/up + down launches)",
-        "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
-        "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
-        "kernel_ms_per_step": round(ffn_ms, 4),
-        "roof_ms_per_step": round(max(t_hbm, t_flop) * 1e3, 4),
-        "frac_of_roof": round(max(t_hbm, t_flop) / ffn_s, 4),
-    })
-
-    clocks = clk.summary() if rank == 0 else None
+    nbytes = roof["algorithmic_bytes"]
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -420,16 +550,32 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": cfg.w_dtype, "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "tokens_per_rank_per_step": tokens_per_step,
                    "layers": cfg.layers, "parallelism": f"dp{world} replicas (no collective)",
+                   "act_dtype": act_dtype,
                    "l2": "inputs larger than L2: %.1f GB of expert weights per step" % (nbytes / 1e9)},
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": int(launches),
-        "clocks": clocks,
+        "clocks": clocks if rank == 0 else None,
     }
     if merge_info is not None:
         out["split_weight"] = merge_info
     if prefetch_info is not None:
         out["prefetch"] = prefetch_info
+
+    # ---- further workloads in the same run (one GPU only)
+    if world == 1 and args.workloads.strip():
+        del dls, pipe, step, xs
+        import gc
+        gc.collect()
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        extra = {}
+        for w in args.workloads.split(","):
+            w = int(w)
+            if w == args.config:
+                continue
+            extra[config(w).name] = measure_extra_workload(w, args, dev, stream, peaks, peak_src)
+        out["workloads"] = extra
     return out, cfg
 
 
@@ -579,9 +725,67 @@ def run_reference(args, rank, world):
     }
 
 
+# ----------------------------------------------------------------------- peaks
+def measure_peaks(reps: int = 10):
+    """Denominators the driver's peak file does not carry, measured with
+    library kernels on this GPU (CUDA events, best of `reps` after warm-up,
+    no clock changes): the dense fp8 e4m3 GEMM (torch._scaled_mm at 8192^3,
+    unit scales, bf16 out), the dense bf16 GEMM beside it (same shape), and
+    the read-only HBM stream (torch.sum over 4 GiB of fp32) beside a copy."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+
+    def best(fn, warm=3):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return min(ts)
+
+    n = 8192
+    out = {}
+    with ClockSampler(0) as clk:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()   # column-major
+        one = torch.ones((), device=dev)
+        ms = best(lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16))
+        out["fp8_tflops"] = round(2.0 * n ** 3 / (ms * 1e-3) / 1e12, 1)
+        del a, b
+        a16 = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+        b16 = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+        ms = best(lambda: torch.matmul(a16, b16))
+        out["bf16_tflops_same_run"] = round(2.0 * n ** 3 / (ms * 1e-3) / 1e12, 1)
+        del a16, b16
+        x = torch.rand(1 << 30, device=dev)                       # 4 GiB fp32
+        ms = best(lambda: x.sum())
+        out["hbm_read_gbs"] = round(x.numel() * 4 / (ms * 1e-3) / 1e9, 1)
+        y = torch.empty_like(x)
+        ms = best(lambda: y.copy_(x))
+        out["hbm_copy_gbs_same_run"] = round(2 * x.numel() * 4 / (ms * 1e-3) / 1e9, 1)
+        del x, y
+        torch.cuda.synchronize()
+    out["clocks"] = clk.summary()
+    out["method"] = ("CUDA events, best of %d after 3 warm-up calls; fp8: torch._scaled_mm "
+                     "e4m3 x e4m3 8192^3, unit fp32 scales, bf16 out; bf16: torch.matmul "
+                     "8192^3; read: torch.sum over 2^30 fp32; copy: Tensor.copy_ of 4 GiB "
+                     "(read + write bytes)" % reps)
+    return out
+
+
 # ----------------------------------------------------------------------- main
 def main(argv=None):
     args = parse_args(argv)
+    if args.measure_peaks:
+        print(json.dumps(measure_peaks()), flush=True)
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -143,8 +143,14 @@ MOE_API moe_status moe_route(const moe_route_cfg *cfg, const void *x, moe_dtype 
  * [H/128, rows] fp32 (one row of scales per 128-column block, so a block's
  * scales for consecutive rows are contiguous): per row and 128 columns
  * s = amax/448, code = e4m3(v/s).
- * topk_idx entries must lie in [0, E) (checked on the device: an entry
- * outside sets the device error word, MOE_ERR_DEVICE_CHECK, and is skipped).
+ * topk_idx entries must lie in [0, E).  This is checked on the device: an
+ * entry outside sets the device error word (moe_check_device() then returns
+ * MOE_ERR_DEVICE_CHECK) and is skipped.  A skipped assignment has no row:
+ * offsets[E] is then less than T*k, its inv_pos entry is -1, the rows
+ * offsets[E] .. T*k-1 of perm_src are left unwritten and the same rows of
+ * x_perm hold no defined value.  The gather checks every perm_src value
+ * against [0, T) before it reads x: a value outside is reported the same way
+ * and its row is zero-filled, so x is never read out of bounds.
  * Limits: H % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.
  * ---------------------------------------------------------------------- */
 MOE_API size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
@@ -163,10 +169,13 @@ MOE_API moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const
  * allowed.
  *
  * Same arguments and results as moe_permute without (workspace,
- * workspace_bytes): the scratch lives in a fixed 1 MiB array inside the
- * library's device memory, which every GPU that loads the library holds until
- * the process exits.  It allocates nothing (no cudaMalloc, cudaFree or
- * allocating library call).
+ * workspace_bytes): the scratch lives in a fixed 1 MiB array in the
+ * library's device code module.  CUDA places it on a device when it loads
+ * that module there (with the default lazy module loading, at the first
+ * permutation call or symbol lookup on that device, not when the library is
+ * opened); from then on that GPU holds it until the process exits.  The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ * Arguments are checked as in moe_permute before any CUDA call is made.
  *   - Limit: moe_permute_workspace_size(T, k, E) <= 1 MiB, i.e.
  *     8 * ceil(T*k / 2048) * E bytes (E = 256: up to 1,048,576 token-expert
  *     assignments).  Larger sizes return MOE_ERR_WORKSPACE and enqueue nothing.
@@ -225,14 +234,27 @@ typedef struct moe_expert_table {
  * For every routed expert e with n_e = offsets[e+1] - offsets[e] > 0 and,
  * when has_shared, for the shared expert on rows T*k .. T*k+T-1:
  *   G = X_e W_gu[e]^T                     X_e = x_perm rows of e
- *   h = silu(G[:, :I]) * G[:, I:]         -> h rows of e   (bf16)
+ *   h = silu(G[:, :I]) * G[:, I:]         -> h rows of e   (act_dtype)
  *   y = h W_down[e]^T                     -> y_perm rows of e (bf16)
  * fp32 accumulation on the tensor cores.
  * x_perm  [rows, H] act_dtype (rows = T*k + (has_shared ? T : 0)).
- * h       [rows, I] bf16 (intermediate, caller-owned).
+ * h       [rows, I] act_dtype (intermediate, caller-owned).
  * y_perm  [rows, H] bf16 out.
- * Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024; w_dtype MOE_BF16 with
- * act_dtype MOE_BF16, or w_dtype MOE_E4M3 with act_dtype MOE_BF16.
+ * Supported (w_dtype, act_dtype):
+ *   MOE_BF16 / MOE_BF16  bf16 weights and activations, bf16 tensor-core MMA.
+ *   MOE_E4M3 / MOE_BF16  e4m3 weights (code x fp32 128x128 block scale), bf16
+ *                        activations: the weights are dequantised to bf16 in
+ *                        shared memory and the bf16 MMA runs.
+ *   MOE_E4M3 / MOE_E4M3  both GEMMs on the fp8 tensor cores.  x_perm is e4m3
+ *                        with x_perm_scales [H/128, rows] fp32 as moe_permute
+ *                        writes them (x = code x scale per row and 128
+ *                        columns); h is e4m3 [rows, I] and its scales
+ *                        [I/128, rows] fp32 go to the workspace, which must
+ *                        hold moe_grouped_ffn_workspace_size(d) bytes.
+ *                        Requires H % 256 == 0.
+ * x_perm_scales and the workspace are ignored (may be NULL, size 0) in the
+ * two bf16-activation combinations.
+ * Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.
  * ---------------------------------------------------------------------- */
 typedef struct moe_ffn_desc {
     int32_t T, H, I, E, k;

@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kThreads) k_scatter(const int32_t* __restrict_
             for (int w = 0; w < warp; ++w) pos += wcnt[w * E + e];
             perm_src[pos] = static_cast<int32_t>(a / k);
             inv_pos[a] = pos;
+        } else if (a < A) {
+            inv_pos[a] = -1;  // skipped (reported): the combine sees no row
         }
         __syncthreads();
         if (e >= 0 && leader) {
@@ -145,18 +147,37 @@ __device__ __forceinline__ void load8(const float* row, int c, float (&v)[8]) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+// Source token of permuted row r, or -1 when it is not a token of x.  Rows
+// r < A come from perm_src; when an expert index was skipped (out of range)
+// the rows past the last scattered one were never written, so the value is
+// checked before it addresses x.
+__device__ __forceinline__ int64_t gather_source(const int32_t* perm_src, int64_t r, int64_t A,
+                                                 int64_t T, int* err) {
+    if (r >= A) return r - A;
+    const int64_t src = perm_src[r];
+    if (src < 0 || src >= T) {
+        if ((threadIdx.x & 31) == 0) atomicOr(err, kDevErrIndex);
+        return -1;
+    }
+    return src;
+}
+
 // One warp per output row; 8 columns (one 16-byte bf16 vector) per lane step.
 template <typename XT>
 __global__ void __launch_bounds__(256) k_gather_bf16(const XT* __restrict__ x,
                                                      const int32_t* __restrict__ perm_src,
-                                                     int64_t A, int64_t rows, int H,
-                                                     __nv_bfloat16* __restrict__ out) {
+                                                     int64_t A, int64_t T, int64_t rows, int H,
+                                                     __nv_bfloat16* __restrict__ out, int* err) {
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= rows) return;
     const int lane = threadIdx.x & 31;
-    const int64_t src = r < A ? perm_src[r] : r - A;
-    const XT* in = x + src * H;
+    const int64_t src = gather_source(perm_src, r, A, T, err);
     __nv_bfloat16* o = out + r * H;
+    if (src < 0) {  // reported above: the row is zero-filled
+        for (int c = lane * 8; c < H; c += 256) *reinterpret_cast<uint4*>(o + c) = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const XT* in = x + src * H;
     for (int c = lane * 8; c < H; c += 256) {
         if constexpr (sizeof(XT) == 2) {
             *reinterpret_cast<uint4*>(o + c) = *reinterpret_cast<const uint4*>(in + c);
@@ -172,39 +193,60 @@ __global__ void __launch_bounds__(256) k_gather_bf16(const XT* __restrict__ x,
     }
 }
 
-// One warp per output row; per 128 columns: s = amax / 448, code = e4m3(v / s).
+// Eight consecutive values of a bf16 or fp32 row as fp32: one or two 16-byte loads.
+__device__ __forceinline__ void load8(const __nv_bfloat16* row, int c, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(row + c);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+// One warp per output row, two 128-column blocks per step: lanes 0-15 hold
+// block b and lanes 16-31 block b + 1, 8 columns per lane (16-byte loads,
+// 8-byte stores).  Per block: s = amax / 448, code = e4m3(v / s).
 template <typename XT>
 __global__ void __launch_bounds__(256) k_gather_e4m3(const XT* __restrict__ x,
                                                      const int32_t* __restrict__ perm_src,
-                                                     int64_t A, int64_t rows, int H,
+                                                     int64_t A, int64_t T, int64_t rows, int H,
                                                      uint8_t* __restrict__ out,
-                                                     float* __restrict__ scales) {
+                                                     float* __restrict__ scales, int* err) {
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= rows) return;
     const int lane = threadIdx.x & 31;
-    const int64_t src = r < A ? perm_src[r] : r - A;
-    const XT* in = x + src * H;
-    for (int c0 = 0; c0 < H; c0 += 128) {
-        float v[4];
+    const int64_t src = gather_source(perm_src, r, A, T, err);
+    const XT* in = x + (src < 0 ? 0 : src) * H;
+    const int nblk = H / 128;
+    for (int b0 = 0; b0 < nblk; b0 += 2) {
+        const int b = b0 + (lane >> 4);
+        const bool act = b < nblk;
+        const int c = b * 128 + (lane & 15) * 8;
+        float v[8];
+        if (act && src >= 0) {
+            load8(in, c, v);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if constexpr (sizeof(XT) == 2)
-                v[i] = __bfloat162float(in[c0 + lane * 4 + i]);
-            else
-                v[i] = in[c0 + lane * 4 + i];
+            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
         }
-        float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+        float m = 0.0f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const float s = (m > 0.0f) ? m / 448.0f : 1.0f;
-        uint32_t packed = 0;
+        uint32_t packed[2] = {0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 8; ++i) {
             const float q = fminf(fmaxf(v[i] / s, -448.0f), 448.0f);
-            packed |= (uint32_t)__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3) << (8 * i);
+            packed[i >> 2] |= (uint32_t)__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3) << (8 * (i & 3));
         }
-        *reinterpret_cast<uint32_t*>(out + r * H + c0 + lane * 4) = packed;
-        if (lane == 0) scales[(int64_t)(c0 / 128) * rows + r] = s;  // [H/128][rows]
+        if (act) {
+            *reinterpret_cast<uint2*>(out + r * H + c) = make_uint2(packed[0], packed[1]);
+            if ((lane & 15) == 0) scales[(int64_t)b * rows + r] = s;  // [H/128][rows]
+        }
     }
 }
 
@@ -223,11 +265,17 @@ size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E) {
     return (size_t)(2 * nb * E) * sizeof(int32_t);
 }
 
-moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t* topk_idx,
-                       const void* x, moe_dtype x_dtype, moe_dtype perm_dtype, int32_t with_shared,
-                       int32_t* offsets, int32_t* perm_src, int32_t* inv_pos, void* x_perm,
-                       float* x_perm_scales, void* workspace, size_t workspace_bytes,
-                       cudaStream_t stream) {
+}  // extern "C"
+
+namespace swb {
+namespace {
+
+// Host-side checks shared by moe_permute and moe_permute_noalloc: everything
+// but the workspace, before anything is enqueued or any CUDA call is made.
+moe_status permute_check_args(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t* topk_idx,
+                              const void* x, moe_dtype x_dtype, moe_dtype perm_dtype,
+                              int32_t* offsets, int32_t* perm_src, int32_t* inv_pos, void* x_perm,
+                              float* x_perm_scales) {
     if (T < 0 || k <= 0 || k > MOE_MAX_TOPK || E <= 0 || E > MOE_MAX_EXPERTS || H <= 0 ||
         H % 128)
         return fail(MOE_ERR_INVALID_ARG, "moe_permute: T=%d k=%d E=%d H=%d", T, k, E, H);
@@ -236,9 +284,7 @@ moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t
     if (perm_dtype != MOE_BF16 && perm_dtype != MOE_E4M3)
         return fail(MOE_ERR_UNSUPPORTED, "moe_permute: x_perm dtype %d", (int)perm_dtype);
     if (!offsets) return fail(MOE_ERR_INVALID_ARG, "moe_permute: offsets is NULL");
-    const int64_t A = (int64_t)T * k;
-    const int64_t rows = A + (with_shared ? T : 0);
-    if (A + T > INT32_MAX) return fail(MOE_ERR_UNSUPPORTED, "moe_permute: too many rows");
+    if ((int64_t)T * k + T > INT32_MAX) return fail(MOE_ERR_UNSUPPORTED, "moe_permute: too many rows");
     if (T > 0 && (!topk_idx || !x || !perm_src || !inv_pos))
         return fail(MOE_ERR_INVALID_ARG, "moe_permute: NULL pointer");
     if (perm_dtype == MOE_E4M3 && T > 0 && x_perm && !x_perm_scales)
@@ -247,12 +293,30 @@ moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t
         !aligned(perm_src, 16) || !aligned(inv_pos, 16) || !aligned(x_perm, 16) ||
         !aligned(x_perm_scales, 16))
         return fail(MOE_ERR_INVALID_ARG, "moe_permute: pointers must be 16-byte aligned");
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace swb
+
+extern "C" {
+
+moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t* topk_idx,
+                       const void* x, moe_dtype x_dtype, moe_dtype perm_dtype, int32_t with_shared,
+                       int32_t* offsets, int32_t* perm_src, int32_t* inv_pos, void* x_perm,
+                       float* x_perm_scales, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+    moe_status st = permute_check_args(T, k, E, H, topk_idx, x, x_dtype, perm_dtype, offsets,
+                                       perm_src, inv_pos, x_perm, x_perm_scales);
+    if (st != MOE_OK) return st;
+    const int64_t A = (int64_t)T * k;
+    const int64_t rows = A + (with_shared ? T : 0);
     const size_t need = moe_permute_workspace_size(T, k, E);
     if (workspace_bytes < need || (need && !workspace))
         return fail(MOE_ERR_WORKSPACE, "moe_permute: workspace %zu < %zu bytes",
                     workspace_bytes, need);
     int* err = nullptr;
-    moe_status st = device_error_word(&err);
+    st = device_error_word(&err);
     if (st != MOE_OK) return st;
     const int64_t nb = num_blocks(A);
     int32_t* blk_counts = static_cast<int32_t*>(workspace);
@@ -274,21 +338,22 @@ moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t
         if (perm_dtype == MOE_BF16) {
             if (x_dtype == MOE_BF16)
                 k_gather_bf16<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
-                                                     perm_src, A, rows, H,
-                                                     static_cast<__nv_bfloat16*>(x_perm));
+                                                     perm_src, A, T, rows, H,
+                                                     static_cast<__nv_bfloat16*>(x_perm), err);
             else
                 k_gather_bf16<<<g, 256, 0, stream>>>(static_cast<const float*>(x), perm_src, A,
-                                                     rows, H,
-                                                     static_cast<__nv_bfloat16*>(x_perm));
+                                                     T, rows, H,
+                                                     static_cast<__nv_bfloat16*>(x_perm), err);
         } else {
             if (x_dtype == MOE_BF16)
                 k_gather_e4m3<<<g, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x),
-                                                     perm_src, A, rows, H,
-                                                     static_cast<uint8_t*>(x_perm), x_perm_scales);
+                                                     perm_src, A, T, rows, H,
+                                                     static_cast<uint8_t*>(x_perm), x_perm_scales,
+                                                     err);
             else
                 k_gather_e4m3<<<g, 256, 0, stream>>>(static_cast<const float*>(x), perm_src, A,
-                                                     rows, H, static_cast<uint8_t*>(x_perm),
-                                                     x_perm_scales);
+                                                     T, rows, H, static_cast<uint8_t*>(x_perm),
+                                                     x_perm_scales, err);
         }
         SWB_LAUNCHED("moe_permute: gather kernel");
     }
@@ -307,8 +372,10 @@ moe_status moe_permute(int32_t T, int32_t k, int32_t E, int32_t H, const int32_t
 // path where a cudaMalloc (which may synchronise the whole device) is not
 // allowed.  The scratch that moe_permute takes as `workspace` (per-block
 // expert counts and bases) lives instead in a fixed array in this library's
-// device memory, created when the library is loaded and held by every GPU
-// that loads it until the process exits.
+// device memory.  The array belongs to this file's device code module: it is
+// placed on a device when that module is loaded there (with CUDA's default
+// lazy loading, at the first kernel launch or symbol lookup of this file on
+// that device) and stays until the process exits.
 // ---------------------------------------------------------------------------
 namespace swb {
 namespace {
@@ -352,6 +419,9 @@ moe_status moe_permute_noalloc(int32_t T, int32_t k, int32_t E, int32_t H,
                                moe_dtype perm_dtype, int32_t with_shared, int32_t* offsets,
                                int32_t* perm_src, int32_t* inv_pos, void* x_perm,
                                float* x_perm_scales, cudaStream_t stream) {
+    moe_status st = permute_check_args(T, k, E, H, topk_idx, x, x_dtype, perm_dtype, offsets,
+                                       perm_src, inv_pos, x_perm, x_perm_scales);
+    if (st != MOE_OK) return st;
     const size_t need = moe_permute_workspace_size(T, k, E);
     if (need > kPermuteScratchBytes)
         return fail(MOE_ERR_WORKSPACE,
@@ -359,7 +429,7 @@ moe_status moe_permute_noalloc(int32_t T, int32_t k, int32_t E, int32_t H,
                     "the built-in %zu bytes (use moe_permute with a workspace)",
                     T, k, E, need, kPermuteScratchBytes);
     void* scratch = nullptr;
-    moe_status st = permute_scratch_address(&scratch);
+    st = permute_scratch_address(&scratch);
     if (st != MOE_OK) return st;
     // Every scratch word the kernels read is written earlier in the same
     // call (block counts, then bases), so nothing needs clearing first.

@@ -23,6 +23,22 @@ MID_FP8 = config(5).with_(cfg_id=24, name="mid_fp8_T300_H512_I256_E32", T=300, H
                           E=32, k=4, n_group=4, topk_group=2, local_count=8, layers=1)
 DECODE_FP8 = config(5).with_(cfg_id=25, name="decode_fp8_T7_H256_I128_E64", T=7, H=256, I=128,
                              E=64, k=8, n_group=8, topk_group=4, local_count=16, layers=1)
+# Mid-size layers (whole-layer, element-by-element against the oracle) that
+# reach each token-tile width of the grouped GEMMs with ragged tiles:
+#   ~256 tokens per expert -> 256-token tiles (one 512-column TMEM set, 16
+#   epilogue warps for bf16 weights, 8 with e4m3 weights);
+#   ~125 tokens per expert -> 128-token tiles, double-buffered accumulators,
+#   row counts that are not multiples of 16.
+MID_BN256 = config(2).with_(cfg_id=27, name="mid_bn256_T2048_H512_I256_E8_k1", T=2048, H=512,
+                            I=256, E=8, k=1, n_group=1, topk_group=1, local_count=3)
+MID_BN256_FP8 = config(5).with_(cfg_id=28, name="mid_bn256_fp8_T2048_H512_I256_E8_k1", T=2048,
+                                H=512, I=256, E=8, k=1, n_group=1, topk_group=1, local_count=3,
+                                layers=1)
+MID_BN128 = config(2).with_(cfg_id=29, name="mid_bn128_T1000_H384_I256_E16_k2", T=1000, H=384,
+                            I=256, E=16, k=2, n_group=4, topk_group=2, local_count=5)
+MID_BN128_FP8 = config(5).with_(cfg_id=30, name="mid_bn128_fp8_T1000_H512_I256_E16_k2", T=1000,
+                                H=512, I=256, E=16, k=2, n_group=4, topk_group=2, local_count=5,
+                                layers=1)
 # the largest shapes the ABI takes: 1024 experts, k = 32, 32 groups (one per lane)
 MAX_EXPERTS = config(2).with_(cfg_id=26, name="max_E1024_k32_G32_T64", T=64, H=256, I=128,
                               E=1024, k=32, n_group=32, topk_group=4, local_count=256)

@@ -15,8 +15,9 @@ from moe_inputs import config, device as mdev, gen
 from oracle import workload as ow
 from split_weight_b200 import _lib as L
 
-from gpu_util import (DECODE_FP8, MAX_EXPERTS, MID_FP8, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16,
-                      RTOL_FP8, SPARSE_DECODE, assert_close_rel, run_layer, sync_check, to_np)
+from gpu_util import (DECODE_FP8, MAX_EXPERTS, MID_BN128, MID_BN128_FP8, MID_BN256, MID_BN256_FP8,
+                      MID_FP8, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16, RTOL_FP8,
+                      SPARSE_DECODE, assert_close_rel, run_layer, sync_check, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -64,6 +65,9 @@ def _rtol(cfg):
 
 @pytest.mark.parametrize("cfg", SMALL + [MID_FP8, DECODE_FP8, MAX_EXPERTS], ids=lambda c: c.name)
 def test_small_layer_full_parity(cfg):
+    """Whole layers, every output element against the oracle.  The e4m3-weight
+    workloads run their stated path: bf16 activations, the weights
+    dequantised to bf16 in shared memory, the bf16 tensor-core MMA."""
     dl = mdev.build_layer(cfg)
     run_layer(dl)
     y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
@@ -72,16 +76,35 @@ def test_small_layer_full_parity(cfg):
     assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
 
 
-@pytest.mark.parametrize("cfg", [MID_FP8, DECODE_FP8], ids=lambda c: c.name)
-def test_fp8_weights_with_bf16_activations(cfg):
-    """The conversion path: e4m3 weights dequantised to bf16 in shared memory,
-    bf16 activations, bf16 tensor-core MMA."""
-    dl = mdev.build_layer(cfg, act_dtype="bf16")
+@pytest.mark.parametrize("cfg", [MID_BN256, MID_BN256_FP8, MID_BN128, MID_BN128_FP8],
+                         ids=lambda c: c.name)
+def test_mid_layer_each_tile_width_full_parity(cfg):
+    """Whole mid-size layers whose experts get ~256 or ~125 tokens each, so
+    the grouped GEMMs run 256-token tiles (one 512-column TMEM accumulator
+    set, the wide epilogue) or 128-token tiles with ragged row counts;
+    every output element against the oracle."""
+    dl = mdev.build_layer(cfg)
     run_layer(dl)
     y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
     _check_routing(dl, idx_ref, w_ref)
     _check_permutation(dl, idx_ref)
-    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, RTOL_FP8, f"{cfg.name} y (bf16 act)")
+    counts = np.diff(dl.layer.offsets.cpu().numpy())
+    mean = -(-cfg.A // cfg.E)
+    assert (mean > 160) if cfg.k == 1 else (32 < mean <= 160), "tile width not reached"
+    assert (counts % 16 != 0).any(), "no ragged token tile"
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
+
+
+@pytest.mark.parametrize("cfg", [MID_FP8, DECODE_FP8, MID_BN128_FP8], ids=lambda c: c.name)
+def test_fp8_tensor_core_path_e4m3_activations(cfg):
+    """The opt-in fp8 tensor-core path: x_perm and h quantised to e4m3 per
+    (row, 128 columns), both GEMMs kind::f8f6f4 with per-block promotion."""
+    dl = mdev.build_layer(cfg, act_dtype="e4m3")
+    run_layer(dl)
+    y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
+    _check_routing(dl, idx_ref, w_ref)
+    _check_permutation(dl, idx_ref)
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, RTOL_FP8, f"{cfg.name} y (e4m3 act)")
 
 
 def test_generator_gpu_matches_host(cuda_device):
@@ -163,16 +186,33 @@ def test_kernel_launch_counter(cuda_device):
 
 
 def test_out_of_range_expert_index_is_reported(cuda_device):
+    """An expert index outside [0, E) is skipped and reported.  The rows it
+    leaves unwritten in perm_src hold a value that is not a token (filled
+    here before the call): the gather must check it before reading x, zero
+    the row and report it; the combine must see inv_pos = -1 and skip it."""
     cfg = SPARSE_DECODE
     dl = mdev.build_layer(cfg)
     ml = dl.layer
     h = torch.cuda.current_stream().cuda_stream
     ml.route(dl.x, h)
+    torch.cuda.synchronize()
     ml.topk_idx[0, 0] = cfg.E + 3   # made on the host side: the kernel checks and skips it
+    ml.perm_src.fill_(2**31 - 1)
+    ml.x_perm.fill_(1.0)
     ml.permute(dl.x, h)
     torch.cuda.synchronize()
     assert L.moe_check_device() == L.MOE_ERR_DEVICE_CHECK
     assert L.moe_check_device() == L.MOE_OK   # the word was cleared
+    off = ml.offsets.cpu().numpy()
+    assert off[cfg.E] == cfg.A - 1
+    assert int(ml.inv_pos[0, 0]) == -1
+    assert int(ml.perm_src[cfg.A - 1]) == 2**31 - 1          # never written
+    assert not ml.x_perm[cfg.A - 1].any()                      # zero-filled, not read from x
+    ml.grouped_ffn(h)
+    ml.combine(h)
+    torch.cuda.synchronize()
+    assert L.moe_check_device() == L.MOE_ERR_DEVICE_CHECK     # the combine saw inv_pos = -1
+    assert torch.isfinite(ml.y[:cfg.T].float()).all()
 
 
 # ----------------------------------------------------------------- full size

@@ -5,10 +5,12 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from moe_inputs import config, device as mdev
+from oracle import workload as ow
 from split_weight_b200 import PrefetchPipeline, _lib as L
 
-from gpu_util import MID_SIGMOID, sync_check
+from gpu_util import MID_SIGMOID, RTOL_BF16, assert_close_rel, sync_check, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -24,7 +26,8 @@ def _free_memory(cuda_device):
 def test_pipeline_equals_resident_layers(split):
     """Three layers through two alternate buffers, each filled by
     moe_prefetch_layer from the layer's peer store, give the same bits as
-    each layer computed with its own resident remote pool."""
+    each layer computed with its own resident remote pool, and every output
+    element of every layer, in both passes, matches the CPU oracle."""
     cfg = MID_SIGMOID.with_(cfg_id=17, layers=3)
     dls = [mdev.build_layer(cfg, layer=l) for l in range(cfg.layers)]
     ref = []
@@ -32,6 +35,7 @@ def test_pipeline_equals_resident_layers(split):
         d.layer.forward(d.x)
         ref.append(d.layer.y.clone())
     sync_check()
+    oracle_y = [ow.layer_full(cfg, l, d.pool, d.slot, d.inputs)[0] for l, d in enumerate(dls)]
     stores = [mdev.peer_store(cfg, l, dls[l].layer.weights) for l in range(cfg.layers)]
     for l in range(cfg.layers):   # the peer store holds exactly the remote pool
         assert torch.equal(stores[l], dls[l].layer.weights.remote)
@@ -48,6 +52,48 @@ def test_pipeline_equals_resident_layers(split):
         sync_check()
         for l in range(cfg.layers):
             assert torch.equal(outs[l], ref[l]), f"pass {rep} layer {l}"
+            assert_close_rel(to_np(outs[l][:cfg.T]), oracle_y[l], RTOL_BF16,
+                             f"pass {rep} layer {l} against the oracle")
+
+
+@pytest.mark.parametrize("split", [True], ids=["split"])
+def test_imbalanced_prefill_full_size_through_the_pipeline(split, cuda_device):
+    """The full-size imbalanced prefill (2 layers x 16384 tokens, Zipf-skewed
+    routing) run as the benchmark runs it: remote experts only in the peer
+    stores, fetched by moe_prefetch_layer into the two alternate buffers.
+    Routing and permutation bit-exact, sampled output rows of both layers in
+    both passes against the oracle."""
+    cfg = config(4)
+    dls = [mdev.build_layer(cfg, layer=l) for l in range(cfg.layers)]
+    stores = [mdev.peer_store(cfg, l, dls[l].layer.weights) for l in range(cfg.layers)]
+    w0 = dls[0].layer.weights
+    rbytes = w0.n_remote * w0.stride
+    for d in dls:   # the pipeline's buffers replace the layers' own remote pools
+        d.layer.weights.remote = torch.empty(1, dtype=torch.uint8, device=cuda_device)
+    gc.collect()
+    torch.cuda.empty_cache()
+    pipe = PrefetchPipeline([d.layer for d in dls], stores, rbytes, split=split)
+    pipe.prime()
+    rng = np.random.default_rng(7)
+    toks = [np.sort(rng.choice(cfg.T, size=5, replace=False)) for _ in range(cfg.layers)]
+    refs, cache = [], {}
+    for l, d in enumerate(dls):
+        idx_ref, w_ref, _ = ow.route(cfg, l, d.inputs)
+        refs.append((idx_ref, w_ref, ow.layer_tokens(cfg, l, toks[l], idx_ref, w_ref, d.pool,
+                                                     d.slot, d.inputs, cache)))
+        cache.clear()
+    for rep in range(2):
+        outs = pipe.run([d.x for d in dls])
+        sync_check()
+        for l, d in enumerate(dls):
+            idx_ref, w_ref, y_ref = refs[l]
+            np.testing.assert_array_equal(d.layer.topk_idx[:cfg.T].cpu().numpy(), idx_ref)
+            off, src, inv = oracle.permute(idx_ref, cfg.E)
+            np.testing.assert_array_equal(d.layer.offsets.cpu().numpy(), off)
+            np.testing.assert_array_equal(d.layer.inv_pos[:cfg.T].cpu().numpy(), inv)
+            y = to_np(outs[l][torch.from_numpy(toks[l]).to(cuda_device)])
+            assert_close_rel(y, y_ref, RTOL_BF16, f"pass {rep} layer {l} sampled rows")
+    del pipe, stores, dls
 
 
 def test_wait_ready_times_out_then_completes(cuda_device):

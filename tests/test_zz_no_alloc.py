@@ -69,3 +69,14 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
                                None, None)
     assert rc == L.MOE_ERR_WORKSPACE
     assert "built-in" in L.moe_last_error()
+
+
+def test_noalloc_checks_arguments_before_any_cuda_call():
+    # a bad hidden size (not a multiple of 128) is an argument error, found on
+    # the host before the scratch array's address is looked up
+    rc = L.moe_permute_noalloc(4, 2, 8, 100, 16, 16, L.MOE_BF16, L.MOE_BF16, 0, 16, 16, 16, None,
+                               None, None)
+    assert rc == L.MOE_ERR_INVALID_ARG
+    rc = L.moe_permute_noalloc(4, 2, 8, 256, 16, 16, L.MOE_E4M3, L.MOE_BF16, 0, 16, 16, 16, None,
+                               None, None)
+    assert rc == L.MOE_ERR_UNSUPPORTED
