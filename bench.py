@@ -53,9 +53,17 @@ def parse_args(argv=None):
     p.add_argument("--act-dtype", choices=["bf16", "e4m3"], default="bf16",
                    help="activations the grouped GEMMs read (e4m3: opt-in fp8 tensor-core path, "
                         "e4m3-weight workloads only)")
-    p.add_argument("--workloads", default="3,5",
+    p.add_argument("--workloads", default="3,4,5",
                    help="further workloads measured in the same run (1 GPU only; '' for none)")
     p.add_argument("--workload-steps", type=int, default=5)
+    p.add_argument("--gate-slots", type=int, default=0,
+                   help="pipelined workloads: per-chunk readiness flags every N remote slots "
+                        "instead of waiting for the whole fetch (0: event-gated)")
+    p.add_argument("--window-inter", type=int, default=12288,
+                   help="intermediate size of the dense block that stands in for the attention "
+                        "block in the prefetch-window measurement (0: skip it)")
+    p.add_argument("--no-schedules", action="store_true",
+                   help="pipelined workloads: measure only the configured prefetch schedule")
     p.add_argument("--measure-peaks", action="store_true",
                    help="measure the fp8 dense GEMM peak and the read-only HBM peak, print JSON")
     return p.parse_args(argv)
@@ -249,7 +257,7 @@ def build_workload(cfg, args, dev, act_dtype):
         stores = [mdev.peer_store(cfg, l, dls[l].layer.weights, dev) for l in range(cfg.layers)]
         rbytes = dls[0].layer.weights.n_remote * dls[0].layer.weights.stride
         pipe = PrefetchPipeline([d.layer for d in dls], stores, rbytes, dev,
-                                split=args.prefetch_split)
+                                split=bool(args.prefetch_split), gate_slots=args.gate_slots)
         for d in dls:  # the layers' own remote pools are not needed: the buffers replace them
             d.layer.weights.remote = torch.empty(1, dtype=torch.uint8, device=dev)
         torch.cuda.empty_cache()
@@ -373,12 +381,16 @@ def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
     c1.record(pipe.copy_stream)
     torch.cuda.synchronize()
     copy_ms = c0.elapsed_time(c1)
-    pipe.g = 0
+    # refill both buffers for the executions that come next (the execution
+    # count keeps growing: readiness epochs must never repeat)
     pipe.prime()
     torch.cuda.synchronize()
     exposed = max(0.0, (piped_ms - nocopy_ms) / cfg.layers)
     return {
-        "schedule": "halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM",
+        "schedule": (("halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM")
+                     + (f"; readiness flags every {pipe.gate_slots} slots" if pipe.gate_slots else
+                        "; compute waits for the whole fetch")
+                     + ("; dense window block" if pipe.window_block is not None else "")),
         "remote_bytes_per_layer": pipe.remote_bytes,
         "copy_alone_ms_per_layer": round(copy_ms, 4),
         "step_ms_pipelined": round(piped_ms, 4),
@@ -386,6 +398,55 @@ def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
         "exposed_copy_ms_per_layer": round(exposed, 4),
         "hidden_fraction": round(1.0 - exposed / copy_ms, 4) if copy_ms > 0 else None,
     }
+
+
+def prefetch_schedules(cfg, pipe, step, stream, args, dev):
+    """Exposed copy time per layer under each prefetch schedule, measured on
+    the same layers and buffers:
+      events_halves   compute waits for each whole fetch, issued in halves
+      flags_whole     the grouped GEMM starts at once and waits per chunk of
+                      8 remote slots on the device (readiness flags); the
+                      fetch is issued whole as soon as its buffer is free
+      flags_halves    the same with the fetch in halves
+      window_*        the same two schedules with a dense compute block
+                      (R1 attention FLOPs) before every MoE block, the
+                      explainer's two-block window; its no-copy baseline runs
+                      the block too
+    Restores the pipeline's own schedule afterwards."""
+    import torch
+    from split_weight_b200 import DenseBlock
+    saved = (pipe.split, pipe.gate_slots, pipe.window_block)
+    steps = max(3, args.workload_steps)
+
+    def run(split, gate_slots, window):
+        torch.cuda.synchronize()
+        pipe.configure(split=split, gate_slots=gate_slots, window_block=window)
+        pipe.prime()
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return prefetch_overlap(cfg, pipe, step, stream, e0.elapsed_time(e1) / steps, steps)
+
+    out = {"events_halves": run(True, 0, None), "flags_whole": run(False, 8, None),
+           "flags_halves": run(True, 8, None)}
+    if args.window_inter > 0:
+        block = DenseBlock(cfg.T, cfg.H, args.window_inter, dev)
+        out["window_block"] = {"inter": args.window_inter,
+                               "flop_per_token": 6.0 * cfg.H * args.window_inter}
+        out["window_events_halves"] = run(True, 0, block)
+        out["window_flags_whole"] = run(False, 8, block)
+        del block
+    torch.cuda.synchronize()
+    pipe.configure(split=saved[0], gate_slots=saved[1], window_block=saved[2])
+    pipe.prime()
+    torch.cuda.synchronize()
+    return out
 
 
 def measure_extra_workload(cfg_id, args, dev, stream, peaks, peak_src):
@@ -416,6 +477,9 @@ def measure_extra_workload(cfg_id, args, dev, stream, peaks, peak_src):
     if pipe is not None:
         out["prefetch"] = prefetch_overlap(cfg, pipe, step, stream,
                                            elapsed_ms / args.workload_steps, args.workload_steps)
+        if not args.no_schedules:
+            out["prefetch"]["schedules"] = prefetch_schedules(cfg, pipe, step, stream, args, dev)
+        L.check(L.moe_check_device())
     del dls, pipe, step
     gc.collect()
     torch.cuda.synchronize()
@@ -462,6 +526,9 @@ def run_ours(args, rank, world, local_rank):
     if pipe is not None:
         prefetch_info = prefetch_overlap(cfg, pipe, step, stream, elapsed_ms / args.steps,
                                          args.steps)
+        if world == 1 and not args.no_schedules:
+            prefetch_info["schedules"] = prefetch_schedules(cfg, pipe, step, stream, args, dev)
+        L.check(L.moe_check_device())
 
     # ---- split-weight ablation: merge both pools into one buffer every step
     merge_info = None

@@ -269,6 +269,34 @@ MOE_API moe_status moe_grouped_ffn(const moe_ffn_desc *d, const moe_expert_table
                            void *y_perm, void *workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
+/* Per-expert readiness (explainer, prefetch caption: the fetch of a layer's
+ * remote experts runs while the rank computes; here the grouped GEMM may
+ * start before the fetch has finished).  With a gate, moe_grouped_ffn_gated
+ * does not need the fetch's ready event: before the first weight load of a
+ * tile of a REMOTE-pool expert in slot s it waits until
+ *   (int32_t)(flags[s / slots_per_flag] - epoch) >= 0
+ * i.e. until moe_prefetch_layer_flagged has landed the chunk that holds s.
+ * Tiles run local experts first, then the shared one, then remote experts in
+ * slot order, the order a fetch fills them in.  The wait polls with a time
+ * limit (timeout_ns; 0 = 2 s); if it runs out the kernels stop early, the
+ * outputs are undefined and moe_check_device() reports MOE_ERR_TIMEOUT.
+ * flags: device, n_flags words, 4-byte aligned, written only by the copy
+ * stream.  A NULL gate (or moe_grouped_ffn) reads the remote pool as it is:
+ * the caller orders the fetch before the call (e.g. with the ready event). */
+typedef struct moe_ready_gate {
+    const uint32_t *flags;
+    uint32_t epoch;
+    int32_t slots_per_flag;  /* remote slots per flag (a flag covers one copy chunk) */
+    int32_t n_flags;         /* >= ceil(remote_count / slots_per_flag) */
+    int64_t timeout_ns;
+} moe_ready_gate;
+
+MOE_API moe_status moe_grouped_ffn_gated(const moe_ffn_desc *d, const moe_expert_table *tbl,
+                                 const moe_ready_gate *gate, const void *x_perm,
+                                 const float *x_perm_scales, const int32_t *offsets, void *h,
+                                 void *y_perm, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Weighted combine (unpermute):
  *   y[t] = sum_{j=0..k-1, ascending} topk_w[t,j] * y_perm[inv_pos[t,j]]
@@ -297,6 +325,89 @@ MOE_API moe_status moe_combine(int32_t T, int32_t k, int32_t H, const void *y_pe
 MOE_API moe_status moe_prefetch_layer(const void *src, void *dst, size_t bytes, size_t chunk_bytes,
                               cudaStream_t copy_stream, cudaEvent_t wait_free,
                               cudaEvent_t ready_out);
+
+/* ------------------------------------------------------------------------
+ * Peer fetch inside a DWDP group (explainer, fetch-path caption: a rank
+ * pulls the experts it lacks from a peer's memory with cudaMemcpyAsync over
+ * NVLink, on the copy engine; contention caption: several destinations can
+ * converge on one source, which time-division multiplexed slicing across
+ * destinations removes).
+ *
+ * A group has G ranks (2 <= G <= 64).  Rank r owns one pool of its experts,
+ * bytes_per_rank bytes (its slots x stride; a multiple of 256).  Its remote
+ * buffer holds the other G-1 pools back to back in rank order, skipping r
+ * (with n experts per rank, rank q owning experts [q*n, q*n+n) in slot
+ * order, expert e of rank q != r sits in slot (q < r ? q : q-1)*n + e - q*n
+ * of rank r's remote buffer).
+ *
+ * The slice plan: each source pool is cut into P = min(slices,
+ * bytes_per_rank/256) pieces, each a multiple of 256 bytes except that the
+ * last takes the rest.  Step j = 0 .. (G-1)*P - 1 of rank r copies piece
+ * floor(j / (G-1)) of source s = (r + 1 + j mod (G-1)) mod G.  At any step j
+ * the map r -> s is the same rotation on every rank, with no fixed point, so
+ * G ranks pulling at the same pace read G different sources: no source ever
+ * serves two destinations in the same step.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_peer_copy {
+    int32_t step;        /* position in the schedule (0-based) */
+    int32_t src_rank;    /* rank whose pool is read */
+    int64_t src_offset;  /* bytes from the start of that pool */
+    int64_t dst_offset;  /* bytes from the start of the remote buffer */
+    int64_t bytes;
+} moe_peer_copy;
+
+/* The plan of `rank` (host only, no CUDA call).  plan == NULL: only
+ * *plan_len is set (a size query).  Otherwise plan must hold plan_capacity
+ * >= *plan_len entries; they are written in step order. */
+MOE_API moe_status moe_peer_fetch_plan(int32_t group_size, int32_t rank, int64_t bytes_per_rank,
+                               int32_t slices, moe_peer_copy *plan, int32_t plan_capacity,
+                               int32_t *plan_len);
+
+/* Enqueues rank's plan on copy_stream: a wait on wait_free (if not NULL),
+ * one cudaMemcpyAsync per step from src_pools[src_rank] + src_offset to
+ * dst + dst_offset, and a record of ready_out (if not NULL).
+ * src_pools: HOST array of G device pointers, the pools of the group's ranks
+ * as this process addresses them (peer access or moe_pool_import);
+ * src_pools[rank] is not read.  dst: (G-1) * bytes_per_rank bytes, 256-byte
+ * aligned, on this rank's device.  Pools must be 256-byte aligned and must
+ * not overlap dst.  No kernel reads a peer's memory: only the copy engine
+ * does. */
+MOE_API moe_status moe_prefetch_peers(int32_t group_size, int32_t rank, const void *const *src_pools,
+                              int64_t bytes_per_rank, int32_t slices, void *dst,
+                              cudaStream_t copy_stream, cudaEvent_t wait_free,
+                              cudaEvent_t ready_out);
+
+/* Lets the current device read peer_device's memory (one process driving
+ * several GPUs).  Already enabled is not an error; MOE_ERR_UNSUPPORTED when
+ * the pair has no peer path. */
+MOE_API moe_status moe_enable_peer_access(int32_t peer_device);
+
+/* One process per GPU: a rank exports its pool, every other rank imports it.
+ * The handle names the CUDA allocation that contains `base` (cudaMalloc'd,
+ * e.g. by a caching allocator) and base's offset inside it. */
+typedef struct moe_pool_handle {
+    char ipc[64];    /* cudaIpcMemHandle_t of the allocation */
+    int64_t offset;  /* bytes from the allocation start to the pool */
+} moe_pool_handle;
+
+MOE_API moe_status moe_pool_export(const void *base, moe_pool_handle *out);
+/* Maps an exported pool into this process: *base_out is the pool, and
+ * *mapping_out the mapping to pass to moe_pool_close once no copy reads it. */
+MOE_API moe_status moe_pool_import(const moe_pool_handle *h, void **base_out, void **mapping_out);
+MOE_API moe_status moe_pool_close(void *mapping);
+
+/* moe_prefetch_layer with per-chunk readiness flags for a gated grouped GEMM:
+ * the copy is issued in chunks of chunk_bytes (> 0; the last takes the
+ * rest), and after chunk c the copy stream writes flags[c] = epoch (a stream
+ * memory operation, ordered after the chunk's copy, executed without SMs).
+ * flags: device, ceil(bytes / chunk_bytes) words.  For a remote pool with
+ * slot stride S, chunk_bytes = slots_per_flag * S makes flag c cover slots
+ * [c*slots_per_flag, (c+1)*slots_per_flag).  MOE_ERR_UNSUPPORTED if the
+ * driver does not provide cuStreamWriteValue32. */
+MOE_API moe_status moe_prefetch_layer_flagged(const void *src, void *dst, size_t bytes,
+                                      size_t chunk_bytes, cudaStream_t copy_stream,
+                                      cudaEvent_t wait_free, uint32_t *flags, uint32_t epoch,
+                                      cudaEvent_t ready_out);
 
 /* Host-side poll of an event with a deadline: MOE_OK once it has completed,
  * MOE_ERR_TIMEOUT after timeout_ms milliseconds, MOE_ERR_CUDA on error. */

@@ -46,6 +46,20 @@ class moe_ffn_desc(ctypes.Structure):
                 ("act_dtype", i32), ("has_shared", i32)]
 
 
+class moe_peer_copy(ctypes.Structure):
+    _fields_ = [("step", i32), ("src_rank", i32), ("src_offset", i64), ("dst_offset", i64),
+                ("bytes", i64)]
+
+
+class moe_pool_handle(ctypes.Structure):
+    _fields_ = [("ipc", ctypes.c_char * 64), ("offset", i64)]
+
+
+class moe_ready_gate(ctypes.Structure):
+    _fields_ = [("flags", vp), ("epoch", ctypes.c_uint32), ("slots_per_flag", i32),
+                ("n_flags", i32), ("timeout_ns", i64)]
+
+
 class MoEError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"{status_string(status)}: {msg}")
@@ -73,8 +87,19 @@ _SIGS = {
     "moe_grouped_ffn_workspace_size": ([ctypes.POINTER(moe_ffn_desc)], sz),
     "moe_grouped_ffn": ([ctypes.POINTER(moe_ffn_desc), ctypes.POINTER(moe_expert_table), vp, vp,
                          vp, vp, vp, vp, sz, vp], i32),
+    "moe_grouped_ffn_gated": ([ctypes.POINTER(moe_ffn_desc), ctypes.POINTER(moe_expert_table),
+                               ctypes.POINTER(moe_ready_gate), vp, vp, vp, vp, vp, vp, sz, vp], i32),
+    "moe_prefetch_layer_flagged": ([vp, vp, sz, sz, vp, vp, vp, ctypes.c_uint32, vp], i32),
     "moe_combine": ([i32, i32, i32, vp, vp, vp, i32, vp, i32, vp], i32),
     "moe_prefetch_layer": ([vp, vp, sz, sz, vp, vp, vp], i32),
+    "moe_peer_fetch_plan": ([i32, i32, i64, i32, ctypes.POINTER(moe_peer_copy), i32,
+                             ctypes.POINTER(i32)], i32),
+    "moe_prefetch_peers": ([i32, i32, ctypes.POINTER(vp), i64, i32, vp, vp, vp, vp], i32),
+    "moe_enable_peer_access": ([i32], i32),
+    "moe_pool_export": ([vp, ctypes.POINTER(moe_pool_handle)], i32),
+    "moe_pool_import": ([ctypes.POINTER(moe_pool_handle), ctypes.POINTER(vp), ctypes.POINTER(vp)],
+                        i32),
+    "moe_pool_close": ([vp], i32),
     "moe_wait_ready": ([vp, i32], i32),
     "moe_check_device": ([], i32),
     "moe_debug_fail_next_cuda_calls": ([i32], None),
@@ -114,8 +139,16 @@ moe_permute_noalloc = _lib.moe_permute_noalloc
 moe_expert_layout_get = _lib.moe_expert_layout_get
 moe_grouped_ffn_workspace_size = _lib.moe_grouped_ffn_workspace_size
 moe_grouped_ffn = _lib.moe_grouped_ffn
+moe_grouped_ffn_gated = _lib.moe_grouped_ffn_gated
+moe_prefetch_layer_flagged = _lib.moe_prefetch_layer_flagged
 moe_combine = _lib.moe_combine
 moe_prefetch_layer = _lib.moe_prefetch_layer
+moe_peer_fetch_plan = _lib.moe_peer_fetch_plan
+moe_prefetch_peers = _lib.moe_prefetch_peers
+moe_enable_peer_access = _lib.moe_enable_peer_access
+moe_pool_export = _lib.moe_pool_export
+moe_pool_import = _lib.moe_pool_import
+moe_pool_close = _lib.moe_pool_close
 moe_wait_ready = _lib.moe_wait_ready
 moe_check_device = _lib.moe_check_device
 moe_debug_fail_next_cuda_calls = _lib.moe_debug_fail_next_cuda_calls
@@ -125,3 +158,13 @@ def expert_layout(H: int, I: int, w_dtype: int) -> moe_expert_layout:
     out = moe_expert_layout()
     check(moe_expert_layout_get(H, I, w_dtype, ctypes.byref(out)))
     return out
+
+
+def peer_fetch_plan(group_size: int, rank: int, bytes_per_rank: int, slices: int):
+    """The rank's time-division fetch schedule as a list of moe_peer_copy."""
+    n = i32(0)
+    check(moe_peer_fetch_plan(group_size, rank, bytes_per_rank, slices, None, 0, ctypes.byref(n)))
+    arr = (moe_peer_copy * max(n.value, 1))()
+    check(moe_peer_fetch_plan(group_size, rank, bytes_per_rank, slices, arr, n.value,
+                              ctypes.byref(n)))
+    return list(arr[:n.value])

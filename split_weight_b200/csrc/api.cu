@@ -111,6 +111,29 @@ moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t ra
     return MOE_OK;
 }
 
+using StreamWriteValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+namespace {
+StreamWriteValue32Fn g_write32 = nullptr;
+}
+
+// cuStreamWriteValue32 through the runtime's driver entry point (the 32-bit
+// stream memory operations of the CUDA 12 driver API need no device opt-in).
+moe_status stream_write_value32(StreamWriteValue32Fn* out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_write32) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cuda_injected_failure())
+            return fail(MOE_ERR_CUDA, "cudaGetDriverEntryPoint: injected failure");
+        const cudaError_t e = cudaGetDriverEntryPoint("cuStreamWriteValue32", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+            return fail(MOE_ERR_UNSUPPORTED, "cuStreamWriteValue32 entry point unavailable");
+        g_write32 = reinterpret_cast<StreamWriteValue32Fn>(fn);
+    }
+    *out = g_write32;
+    return MOE_OK;
+}
+
 std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -184,6 +207,42 @@ moe_status moe_prefetch_layer(const void* src, void* dst, size_t bytes, size_t c
         SWB_CUDA(cudaMemcpyAsync(static_cast<char*>(dst) + off,
                                  static_cast<const char*>(src) + off, n,
                                  cudaMemcpyDeviceToDevice, copy_stream));
+    }
+    if (ready_out) SWB_CUDA(cudaEventRecord(ready_out, copy_stream));
+    return MOE_OK;
+}
+
+moe_status moe_prefetch_layer_flagged(const void* src, void* dst, size_t bytes, size_t chunk_bytes,
+                                      cudaStream_t copy_stream, cudaEvent_t wait_free,
+                                      uint32_t* flags, uint32_t epoch, cudaEvent_t ready_out) {
+    if (bytes > 0 && (!src || !dst))
+        return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_flagged: NULL buffer");
+    if (chunk_bytes == 0 || !flags || !aligned(flags, 4))
+        return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_flagged: chunk_bytes > 0 and "
+                    "4-byte aligned flags needed");
+    if (bytes > 0) {
+        const char* s = static_cast<const char*>(src);
+        char* d = static_cast<char*>(dst);
+        if ((s < d + bytes) && (d < s + bytes))
+            return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_flagged: source and destination "
+                        "overlap");
+    }
+    StreamWriteValue32Fn write32 = nullptr;
+    moe_status st = stream_write_value32(&write32);
+    if (st != MOE_OK) return st;
+    if (wait_free) SWB_CUDA(cudaStreamWaitEvent(copy_stream, wait_free, 0));
+    size_t c = 0;
+    for (size_t off = 0; off < bytes; off += chunk_bytes, ++c) {
+        const size_t n = bytes - off < chunk_bytes ? bytes - off : chunk_bytes;
+        SWB_CUDA(cudaMemcpyAsync(static_cast<char*>(dst) + off,
+                                 static_cast<const char*>(src) + off, n,
+                                 cudaMemcpyDeviceToDevice, copy_stream));
+        if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "cuStreamWriteValue32: injected failure");
+        const CUresult r = write32(reinterpret_cast<CUstream>(copy_stream),
+                                   reinterpret_cast<CUdeviceptr>(flags + c), epoch,
+                                   CU_STREAM_WRITE_VALUE_DEFAULT);
+        if (r != CUDA_SUCCESS)
+            return fail(MOE_ERR_CUDA, "cuStreamWriteValue32 failed (CUresult %d)", (int)r);
     }
     if (ready_out) SWB_CUDA(cudaEventRecord(ready_out, copy_stream));
     return MOE_OK;

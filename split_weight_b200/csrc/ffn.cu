@@ -253,9 +253,28 @@ moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, c
                            const float* x_perm_scales, const int32_t* offsets, void* h,
                            void* y_perm, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream) {
+    return moe_grouped_ffn_gated(d, tbl, nullptr, x_perm, x_perm_scales, offsets, h, y_perm,
+                                 workspace, workspace_bytes, stream);
+}
+
+moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* tbl,
+                                 const moe_ready_gate* gate, const void* x_perm,
+                                 const float* x_perm_scales, const int32_t* offsets, void* h,
+                                 void* y_perm, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
     moe_expert_layout lay;
     moe_status st = validate(d, tbl, &lay);
     if (st != MOE_OK) return st;
+    if (gate) {
+        if (!gate->flags || !aligned(gate->flags, 4) || gate->slots_per_flag <= 0 ||
+            gate->timeout_ns < 0)
+            return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_gated: gate needs flags (4-byte "
+                        "aligned), slots_per_flag > 0 and timeout_ns >= 0");
+        if (gate->n_flags < (tbl->remote_count + gate->slots_per_flag - 1) / gate->slots_per_flag)
+            return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_gated: %d flags cannot cover %d "
+                        "remote slots at %d per flag", gate->n_flags, tbl->remote_count,
+                        gate->slots_per_flag);
+    }
     if (d->T == 0) return MOE_OK;
     if (!x_perm || !offsets || !h || !y_perm)
         return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn: NULL pointer");
@@ -287,6 +306,34 @@ moe_status moe_grouped_ffn(const moe_ffn_desc* d, const moe_expert_table* tbl, c
     a.A = (int32_t)A;
     a.has_shared = d->has_shared ? 1 : 0;
     for (int e = 0; e < d->E; ++e) a.pool_slot[e] = tbl->pool_slot[e];
+    // tile order: local experts by slot, the shared expert, remote experts by
+    // slot (the order a fetch fills the remote buffer in)
+    {
+        static thread_local int32_t by_slot[2][kMaxGroups];
+        for (int q = 0; q < 2; ++q)
+            for (int i = 0; i < kMaxGroups; ++i) by_slot[q][i] = -1;
+        for (int e = 0; e < d->E; ++e) {
+            const uint32_t v = static_cast<uint32_t>(tbl->pool_slot[e]);
+            const int q = (int)(v >> 31), slot = (int)(v & 0x7FFFFFFFu);
+            if (slot < kMaxGroups) by_slot[q][slot] = e;   // slots beyond E: see below
+        }
+        int n = 0;
+        for (int q = 0; q < 2; ++q) {
+            for (int i = 0; i < kMaxGroups && n < d->E + 1; ++i)
+                if (by_slot[q][i] >= 0) a.order[n++] = (uint16_t)by_slot[q][i];
+            if (q == 0 && d->has_shared) a.order[n++] = (uint16_t)d->E;
+        }
+        if (n != G) {  // several experts share a slot, or slots lie beyond kMaxGroups: expert order
+            n = 0;
+            for (int g = 0; g < G; ++g) a.order[n++] = (uint16_t)g;
+        }
+    }
+    if (gate) {
+        a.ready_flags = gate->flags;
+        a.ready_epoch = gate->epoch;
+        a.slots_per_flag = gate->slots_per_flag;
+        a.ready_timeout_ns = gate->timeout_ns > 0 ? (uint64_t)gate->timeout_ns : kWaitLimitNs;
+    }
     const void* base[2] = {tbl->local_base, tbl->remote_base};
     const int32_t count[2] = {tbl->local_count, tbl->remote_count};
     const int64_t stride[2] = {tbl->local_stride, tbl->remote_stride};

@@ -103,11 +103,12 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            int stage = 0;
+            int stage = 0, passed = -1;
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+                if (!gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)) break;
                 const CUtensorMap* wm = &p.w_map[t.map];
                 const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
                 const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
@@ -188,18 +189,20 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         // sits at position j ^ (r % 8).  One 128x128 block scale covers the
         // whole stage (64 columns of K, 128 rows).
         const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. kConvThreads-1
-        int stage = 0;
+        int stage = 0, passed = -1;
         uint32_t phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+            // the block scales sit in the remote buffer too: read them only once landed
+            if (!__all_sync(0xffffffffu, gate_wait(p, t.map, t.slot, passed, abort_flag, p.err))) break;
             const uint8_t* sbase = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map] + p.scale_off;
             const float* sc0 = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
             const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
             const float* sc1 = reinterpret_cast<const float*>(sbase) + (int64_t)rb1 * p.kblocks;
             for (int kb = 0; kb < KB; ++kb) {
-                const float s0 = __ldg(sc0 + (kb >> 1));
-                const float s1 = C::kNA == 2 ? __ldg(sc1 + (kb >> 1)) : 0.0f;
+                const float s0 = __ldcg(sc0 + (kb >> 1));
+                const float s1 = C::kNA == 2 ? __ldcg(sc1 + (kb >> 1)) : 0.0f;
                 ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;

@@ -45,7 +45,21 @@ struct alignas(64) FfnArgs {
     int32_t act_scale_ld;
     uint8_t* out8;
     float* out_scale;
+    // readiness gate of the remote pool (NULL flags: none): the chunk of
+    // slots_per_flag remote slots holding slot s has landed once
+    // ready_flags[s / slots_per_flag] has reached ready_epoch
+    const uint32_t* ready_flags;
+    uint32_t ready_epoch;
+    int32_t slots_per_flag;
+    uint64_t ready_timeout_ns;
+    // tile enumeration order: position i holds group order[i] (local experts
+    // and the shared one first, then the remote experts in slot order, the
+    // order in which a fetch fills them)
+    uint16_t order[kMaxGroups];
 };
+
+// passed by value as a __grid_constant__ kernel parameter (sm_70+ limit 32764 bytes)
+static_assert(sizeof(FfnArgs) <= 32764, "FfnArgs exceeds the kernel parameter limit");
 
 enum { kSingle = 0, kGated = 1, kPair = 2 };
 
@@ -99,13 +113,14 @@ __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
     return t;
 }
 
-// One warp: per-group first row, rows, tile count and (pool, slot), and the
-// exclusive scan of tiles over the groups (routed experts, then the shared one).
+// One warp: per position (group p.order[i]) the first row, rows, tile count
+// and (pool, slot), and the exclusive scan of tiles over the positions.
 template <int BN>
 __device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G, int MT, int lane) {
-    const int per = (G + 31) / 32, g0 = lane * per, g1 = min(G, g0 + per);
+    const int per = (G + 31) / 32, i0 = lane * per, i1 = min(G, i0 + per);
     int sum = 0;
-    for (int g = g0; g < g1; ++g) {
+    for (int i = i0; i < i1; ++i) {
+        const int g = p.order[i];
         int n, r0, ps;
         if (g < p.E) {
             r0 = p.offsets[g];
@@ -117,9 +132,9 @@ __device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G
             n = p.T;
             ps = 2 << 24;
         }
-        tb.row0[g] = r0;
-        tb.n[g] = n;
-        tb.ps[g] = ps;
+        tb.row0[i] = r0;
+        tb.n[i] = n;
+        tb.ps[i] = ps;
         sum += token_tiles<BN>(n) * MT;
     }
     int incl = sum;
@@ -129,11 +144,43 @@ __device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G
         if (lane >= o) incl += v;
     }
     int run = incl - sum;
-    for (int g = g0; g < g1; ++g) {
-        tb.tile_start[g] = run;
-        run += token_tiles<BN>(tb.n[g]) * MT;
+    for (int i = i0; i < i1; ++i) {
+        tb.tile_start[i] = run;
+        run += token_tiles<BN>(tb.n[i]) * MT;
     }
     if (lane == 31) tb.tile_start[G] = incl;
+}
+
+// Per-expert readiness of a fetch still in flight: waits until the chunk of
+// the remote pool that holds `slot` has landed (its flag, written by the copy
+// stream after the chunk, has reached the epoch).  Only remote tiles of a
+// gated call wait.  Every calling thread polls (acquire, GPU scope); the wait
+// gives up after ready_timeout_ns: it raises *abort, sets the timeout bit of
+// the device error word and returns false.  `passed` caches the last flag
+// seen ready by this thread (flags only grow during a call).  On success the
+// async proxy (TMA) is ordered after the acquire.
+__device__ __forceinline__ bool gate_wait(const FfnArgs& p, int map, int slot, int& passed,
+                                          volatile int* abort, int* err) {
+    if (p.ready_flags == nullptr || map != 1) return true;
+    const int f = slot / p.slots_per_flag;
+    if (f == passed) return true;
+    const uint32_t* flag = p.ready_flags + f;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if ((int32_t)(v - p.ready_epoch) >= 0) break;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > p.ready_timeout_ns) {
+            *abort = 1;
+            atomicOr(err, kDevErrTimeout);
+            return false;
+        }
+        __nanosleep(200);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    passed = f;
+    return true;
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }

@@ -96,11 +96,12 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            int stage = 0;
+            int stage = 0, passed = -1;
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+                if (!gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)) break;
                 const CUtensorMap* wm = &p.w_map[t.map];
                 const uint32_t tx = C::kAStage + (uint32_t)t.n_mma * C::kBK8;
                 const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
@@ -176,13 +177,15 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
         float* cu = cg + kC;                 //                              up / row block 1
         float* red_half = scratch + C::kEpiWarps * 2 * kC + part * 2 * 4 * kC;  // [2][4][kC]
         uint32_t tiles_done = 0;
-        int pb = 0;
+        int pb = 0, passed = -1;
         uint32_t use[C::kPBufs];
 #pragma unroll
         for (int b = 0; b < C::kPBufs; ++b) use[b] = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+            // the weight block scales sit in the remote buffer too: read them only once landed
+            if (!__all_sync(0xffffffffu, gate_wait(p, t.map, t.slot, passed, abort_flag, p.err))) break;
             const uint8_t* sbase = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map] + p.scale_off;
             const float* sw0p = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
             const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
             for (int j = 0; j < kC; ++j) acc0[j] = acc1[j] = 0.0f;
             float sx[kSx], sxn[kSx];
             load_sx(0, sx);
-            float sw0 = __ldg(sw0p), sw1 = __ldg(sw1p);
+            float sw0 = __ldcg(sw0p), sw1 = __ldcg(sw1p);
             for (int kb = 0; kb < KB; ++kb) {
 #pragma unroll
                 for (int i = 0; i < kSx; ++i) {
@@ -216,8 +219,8 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
                 float sw0n = 0.0f, sw1n = 0.0f;
                 if (kb + 1 < KB) {   // next block's scales travel while this one is folded in
                     load_sx(kb + 1, sxn);
-                    sw0n = __ldg(sw0p + kb + 1);
-                    sw1n = __ldg(sw1p + kb + 1);
+                    sw0n = __ldcg(sw0p + kb + 1);
+                    sw1n = __ldcg(sw1p + kb + 1);
                 }
                 ok = mbar_wait(smem_u32(&part_full[pb]), use[pb] & 1u, abort_flag, p.err);
                 if (!__all_sync(0xffffffffu, ok)) {

@@ -127,6 +127,21 @@ class SplitWeights:
                                   _ptr(self.shared), self._ps_c)
 
 
+@dataclass
+class ReadyGate:
+    """Per-chunk readiness flags of a remote buffer (moe_ready_gate): flag c
+    covers remote slots [c*slots_per_flag, (c+1)*slots_per_flag) and reaches
+    `epoch` once the copy stream has landed that chunk."""
+    flags: torch.Tensor          # int32 [n_flags] on the device (read as uint32)
+    epoch: int
+    slots_per_flag: int
+    timeout_ns: int = 0          # 0: the library default (2 s)
+
+    def c_struct(self) -> L.moe_ready_gate:
+        return L.moe_ready_gate(self.flags.data_ptr(), self.epoch & 0xFFFFFFFF,
+                                self.slots_per_flag, self.flags.numel(), self.timeout_ns)
+
+
 class MoELayer:
     """One MoE layer with preallocated device buffers."""
 
@@ -175,13 +190,18 @@ class MoELayer:
                               _ptr(self.x_scales),
                               self.perm_ws.data_ptr(), self.perm_ws.numel(), stream))
 
-    def grouped_ffn(self, stream: int, remote: torch.Tensor | None = None) -> None:
+    def grouped_ffn(self, stream: int, remote: torch.Tensor | None = None,
+                    gate: "ReadyGate | None" = None) -> None:
+        """The grouped GEMMs; with a gate, remote experts are read only once
+        their chunk of a fetch still in flight has landed."""
         tbl = self.weights.table(remote)
-        L.check(L.moe_grouped_ffn(ctypes.byref(self._desc), ctypes.byref(tbl),
-                                  self.x_perm.data_ptr(), _ptr(self.x_scales),
-                                  self.offsets.data_ptr(), self.h.data_ptr(),
-                                  self.y_perm.data_ptr(), self.ffn_ws.data_ptr(),
-                                  self.ffn_ws.numel(), stream))
+        g = gate.c_struct() if gate is not None else None
+        L.check(L.moe_grouped_ffn_gated(ctypes.byref(self._desc), ctypes.byref(tbl),
+                                        ctypes.byref(g) if g is not None else None,
+                                        self.x_perm.data_ptr(), _ptr(self.x_scales),
+                                        self.offsets.data_ptr(), self.h.data_ptr(),
+                                        self.y_perm.data_ptr(), self.ffn_ws.data_ptr(),
+                                        self.ffn_ws.numel(), stream))
 
     def combine(self, stream: int) -> None:
         s = self.shape
@@ -218,14 +238,27 @@ class PrefetchPipeline:
     ready is recorded after the second.  Each half then starts in the window
     of routing, permutation and combine between two grouped GEMMs instead of
     the whole fetch running beside the next grouped GEMM.
+
+    With gate_slots > 0 the compute stream does not wait for ready: the fetch
+    writes a readiness flag per chunk of gate_slots remote slots
+    (moe_prefetch_layer_flagged, epoch g + 1 for execution g) and the grouped
+    GEMM of execution g starts at once, running local experts first and
+    waiting on the device, per chunk, for the remote experts it reaches
+    (moe_grouped_ffn_gated).
+
+    window_block(l, x, stream), if given, is enqueued before layer l's MoE
+    block: compute that the fetch also hides behind (the explainer's
+    attention block between two MoE blocks).
     """
 
     def __init__(self, layers: list[MoELayer], peer_stores: list[torch.Tensor],
                  remote_bytes: int, device: torch.device | str = "cuda", chunk_bytes: int = 0,
-                 split: bool = True):
+                 split: bool = True, gate_slots: int = 0, window_block=None,
+                 gate_timeout_ns: int = 0):
         self.layers, self.peer_stores = layers, peer_stores
         self.remote_bytes, self.chunk_bytes = remote_bytes, chunk_bytes
         self.split, self.pending = split, None
+        self.gate_slots, self.window_block, self.gate_timeout_ns = gate_slots, window_block, gate_timeout_ns
         dev = torch.device(device)
         self.bufs = [torch.empty(max(remote_bytes, 1), dtype=torch.uint8, device=dev)
                      for _ in range(2)]
@@ -235,58 +268,108 @@ class PrefetchPipeline:
         for ev in self.ready + self.free:   # torch creates CUDA events on first record
             ev.record(self.copy_stream)
         self.g = 0
+        self.stride = layers[0].weights.stride
+        self.flags = None
+        self.configure(gate_slots=gate_slots)
 
-    def prefetch(self, layer: int, buf: int, wait_free: torch.cuda.Event | None) -> None:
+    def configure(self, split: bool | None = None, gate_slots: int | None = None,
+                  window_block=False) -> None:
+        """Switches the schedule between runs (after a synchronisation: no
+        fetch may be in flight).  window_block=False leaves it as it is."""
+        if split is not None:
+            self.split = split
+        if window_block is not False:
+            self.window_block = window_block
+        if gate_slots is not None:
+            self.gate_slots = gate_slots
+            if gate_slots > 0:
+                assert self.remote_bytes % self.stride == 0
+                n_slots = self.remote_bytes // self.stride
+                self.n_flags = max(1, -(-n_slots // gate_slots))
+                dev = self.bufs[0].device
+                # flags only grow: fresh zeros are below every epoch still to come
+                self.flags = [torch.zeros(self.n_flags, dtype=torch.int32, device=dev)
+                              for _ in range(2)]
+        self.pending = None
+
+    # -- copies -------------------------------------------------------------
+    def _copy(self, layer: int, buf: int, lo: int, hi: int, wait_free, ready, epoch: int) -> None:
+        src = self.peer_stores[layer].data_ptr() + lo
+        dst = self.bufs[buf].data_ptr() + lo
+        wf = wait_free.cuda_event if wait_free is not None else None
+        rd = ready.cuda_event if ready is not None else None
+        if self.gate_slots > 0:
+            chunk = self.gate_slots * self.stride
+            assert lo % chunk == 0
+            L.check(L.moe_prefetch_layer_flagged(src, dst, hi - lo, chunk,
+                                                 self.copy_stream.cuda_stream, wf,
+                                                 self.flags[buf].data_ptr() + 4 * (lo // chunk),
+                                                 epoch & 0xFFFFFFFF, rd))
+        else:
+            L.check(L.moe_prefetch_layer(src, dst, hi - lo, self.chunk_bytes,
+                                         self.copy_stream.cuda_stream, wf, rd))
+
+    def _cut(self) -> int:
+        if self.gate_slots > 0:
+            chunk = self.gate_slots * self.stride
+            return (self.n_flags // 2) * chunk
+        return (self.remote_bytes // 2) // 256 * 256
+
+    def prefetch(self, layer: int, buf: int, wait_free: torch.cuda.Event | None,
+                 execution: int | None = None) -> None:
+        """The whole fetch of `layer` into bufs[buf] for the given execution."""
         assert self.ready[buf].cuda_event != 0 and (wait_free is None or wait_free.cuda_event != 0)
-        L.check(L.moe_prefetch_layer(self.peer_stores[layer].data_ptr(), self.bufs[buf].data_ptr(),
-                                     self.remote_bytes, self.chunk_bytes,
-                                     self.copy_stream.cuda_stream,
-                                     wait_free.cuda_event if wait_free is not None else None,
-                                     self.ready[buf].cuda_event))
+        ex = self.g if execution is None else execution
+        self._copy(layer, buf, 0, self.remote_bytes, wait_free, self.ready[buf], ex + 1)
 
-    def fetch_half(self, layer: int, buf: int, half: int, wait_free: torch.cuda.Event) -> None:
+    def fetch_half(self, layer: int, buf: int, half: int, wait_free: torch.cuda.Event,
+                   execution: int | None = None) -> None:
         """One half of a fetch; the second half records ready[buf]."""
-        cut = (self.remote_bytes // 2) // 256 * 256
+        cut = self._cut()
         lo, hi = (0, cut) if half == 0 else (cut, self.remote_bytes)
         assert wait_free.cuda_event != 0 and self.ready[buf].cuda_event != 0
-        L.check(L.moe_prefetch_layer(self.peer_stores[layer].data_ptr() + lo,
-                                     self.bufs[buf].data_ptr() + lo, hi - lo, self.chunk_bytes,
-                                     self.copy_stream.cuda_stream, wait_free.cuda_event,
-                                     self.ready[buf].cuda_event if half == 1 else None))
+        ex = self.g if execution is None else execution
+        self._copy(layer, buf, lo, hi, wait_free, self.ready[buf] if half == 1 else None, ex + 1)
 
     def prime(self) -> None:
         """Enqueues the fetches of the next two executions (before a run)."""
         n = len(self.layers)
         self.pending = None
         for i in range(2):
-            self.prefetch((self.g + i) % n, (self.g + i) % 2, None)
+            self.prefetch((self.g + i) % n, (self.g + i) % 2, None, self.g + i)
 
+    # -- compute ------------------------------------------------------------
     def run_layer(self, l: int, x: torch.Tensor, stream: torch.cuda.Stream,
                   prefetch: bool = True, wrap: bool = True, ffn_events=None) -> torch.Tensor:
         """One layer execution; ffn_events = (start, end) events around its
         grouped GEMMs, if given."""
         n = len(self.layers)
-        layer, h, b = self.layers[l], stream.cuda_stream, self.g % 2
+        layer, h, b, g = self.layers[l], stream.cuda_stream, self.g % 2, self.g
+        if self.window_block is not None:
+            self.window_block(l, x, stream)
         layer.route(x, h)
         layer.permute(x, h)
-        if prefetch:
+        gate = None
+        if prefetch and self.gate_slots > 0:
+            gate = ReadyGate(self.flags[b], g + 1, self.gate_slots, self.gate_timeout_ns)
+        elif prefetch:
             stream.wait_event(self.ready[b])
         if ffn_events is not None:
             ffn_events[0].record(stream)
-        layer.grouped_ffn(h, self.bufs[b])
+        layer.grouped_ffn(h, self.bufs[b], gate)
         if ffn_events is not None:
             ffn_events[1].record(stream)
         if prefetch and self.split:
             self.free[b].record(stream)
             if self.pending is not None:  # second half of execution g + 1's fetch
-                self.fetch_half(*self.pending, 1, self.free[b])
+                self.fetch_half(*self.pending, 1, self.free[b], g + 1)
                 self.pending = None
             if l + 2 < n or wrap:        # first half of execution g + 2's
-                self.fetch_half((l + 2) % n, b, 0, self.free[b])
+                self.fetch_half((l + 2) % n, b, 0, self.free[b], g + 2)
                 self.pending = ((l + 2) % n, b)
         elif prefetch and (l + 2 < n or wrap):
             self.free[b].record(stream)
-            self.prefetch((l + 2) % n, b, self.free[b])
+            self.prefetch((l + 2) % n, b, self.free[b], g + 2)
         layer.combine(h)
         self.g += 1
         return layer.y
@@ -298,3 +381,80 @@ class PrefetchPipeline:
         the first pass with prefetch."""
         stream = stream if stream is not None else torch.cuda.current_stream()
         return [self.run_layer(l, xs[l], stream, prefetch, wrap) for l in range(len(self.layers))]
+
+
+class DenseBlock:
+    """A dense SwiGLU block on all of a layer's tokens, run through the same
+    grouped GEMM (one expert that every token uses): compute between two MoE
+    blocks for the prefetch to hide behind.  It stands in for the attention
+    block of the explainer's prefetch caption, which this library does not
+    implement; inter = 12288 at H = 7168 gives 6*H*inter = 528 MFLOP per
+    token, about DeepSeek-R1's attention projections plus causal attention
+    over 4K-token sequences.  Its output is not used."""
+
+    def __init__(self, T: int, H: int, inter: int, device, seed: int = 0):
+        self.T, self.H, self.inter = T, H, inter
+        dev = torch.device(device)
+        self.weights = SplitWeights.allocate(H, inter, "bf16", np.zeros(1, dtype=np.int64),
+                                             np.zeros(1, dtype=np.int64), False, dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        w = self.weights.local.view(torch.bfloat16)
+        w.copy_((torch.randn(w.numel(), device=dev, generator=g) * 0.02).to(torch.bfloat16))
+        self.shape = LayerShape(T=T, H=H, I=inter, E=1, k=1, has_shared=False)
+        self._desc = self.shape.ffn_desc()
+        self.offsets = torch.tensor([0, T], dtype=torch.int32, device=dev)
+        self.h = torch.empty(max(T, 1), inter, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(max(T, 1), H, dtype=torch.bfloat16, device=dev)
+
+    def __call__(self, l: int, x: torch.Tensor, stream: torch.cuda.Stream) -> None:
+        assert x.dtype == torch.bfloat16 and x.shape[0] == self.T
+        tbl = self.weights.table()
+        L.check(L.moe_grouped_ffn(ctypes.byref(self._desc), ctypes.byref(tbl), x.data_ptr(), None,
+                                  self.offsets.data_ptr(), self.h.data_ptr(), self.y.data_ptr(),
+                                  None, 0, stream.cuda_stream))
+
+
+class PeerPools:
+    """The expert pools of a DWDP group as this rank addresses them, and the
+    time-division sliced fetch of the ones it lacks (moe_prefetch_peers).
+
+    ``pools[q]`` is the device address of rank q's pool (``bytes_per_rank``
+    bytes): this rank's own tensor, a peer's through peer access, or a pool
+    mapped with ``import_pool``.  The remote buffer receives the other ranks'
+    pools in rank order, skipping this rank."""
+
+    def __init__(self, group_size: int, rank: int, pools: list[int], bytes_per_rank: int,
+                 slices: int = 8):
+        assert len(pools) == group_size
+        self.G, self.rank, self.bytes_per_rank, self.slices = group_size, rank, bytes_per_rank, slices
+        self._pools = (ctypes.c_void_p * group_size)(*[p or None for p in pools])
+
+    def fetch(self, dst: torch.Tensor, copy_stream: torch.cuda.Stream,
+              wait_free: torch.cuda.Event | None = None,
+              ready: torch.cuda.Event | None = None) -> None:
+        assert dst.numel() * dst.element_size() >= (self.G - 1) * self.bytes_per_rank
+        L.check(L.moe_prefetch_peers(self.G, self.rank, self._pools, self.bytes_per_rank,
+                                     self.slices, dst.data_ptr(), copy_stream.cuda_stream,
+                                     wait_free.cuda_event if wait_free is not None else None,
+                                     ready.cuda_event if ready is not None else None))
+
+
+def export_pool(t: torch.Tensor) -> bytes:
+    """IPC handle (bytes) of the pool held by tensor t, for another process."""
+    h = L.moe_pool_handle()
+    L.check(L.moe_pool_export(t.data_ptr(), ctypes.byref(h)))
+    return ctypes.string_at(ctypes.addressof(h), ctypes.sizeof(h))
+
+
+def import_pool(handle: bytes) -> tuple[int, int]:
+    """Maps a pool exported by another process: (pool address, mapping); pass
+    the mapping to close_pool when no copy reads the pool any more."""
+    h = L.moe_pool_handle.from_buffer_copy(handle)
+    base, mapping = ctypes.c_void_p(), ctypes.c_void_p()
+    L.check(L.moe_pool_import(ctypes.byref(h), ctypes.byref(base), ctypes.byref(mapping)))
+    return base.value, mapping.value
+
+
+def close_pool(mapping: int) -> None:
+    L.check(L.moe_pool_close(mapping))

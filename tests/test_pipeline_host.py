@@ -65,7 +65,9 @@ class FakeLayer:
     def permute(self, x, h):
         pass
 
-    def grouped_ffn(self, h, remote):
+    def grouped_ffn(self, h, remote, gate=None):
+        if gate is not None:   # the gated kernel reads each chunk once its flag reached the epoch
+            Log.ops.append(("gate", "compute", gate.flags.owner, gate.epoch))
         Log.ops.append(("ffn", "compute", self.idx, remote.owner))
 
     def combine(self, h):
@@ -83,13 +85,38 @@ def fake_prefetch(src, dst, nbytes, chunk, stream, wait, ready):
     return L.MOE_OK
 
 
-def replay(ops, nbytes):
+def fake_prefetch_flagged(src, dst, nbytes, chunk, stream, wait, flags, epoch, ready):
+    if wait is not None:
+        ev = FakeEvent.by_id[wait]
+        Log.ops.append(("wait", "copy", ev, ev.version))
+    assert src[1] == dst[1] and src[1] % chunk == 0
+    first = src[1] // chunk
+    assert flags[1] == 4 * first
+    for i, lo in enumerate(range(src[1], src[1] + nbytes, chunk)):
+        hi = min(lo + chunk, src[1] + nbytes)
+        Log.ops.append(("copy", "copy", src[0], dst[0], lo, hi))
+        Log.ops.append(("flag", "copy", flags[0], first + i, epoch))
+    if ready is not None:
+        FakeEvent.by_id[ready].record(FakeStream(name="copy"))
+    return L.MOE_OK
+
+
+class FlagBuffer(Buffer):
+    def __init__(self, owner, n):
+        super().__init__(owner)
+        self.n = n
+
+    def numel(self):
+        return self.n
+
+
+def replay(ops, nbytes, n_flags=0):
     """Runs both streams in order, honouring waits; returns (layer, buffer
     contents) for every grouped GEMM in execution order."""
     done = {}  # event id -> highest executed record version
     queues = {s: [o for o in ops if o[1] == s] for s in ("compute", "copy")}
     pos = {s: 0 for s in queues}
-    buffers, seen, moved = {}, [], True
+    buffers, seen, moved, flags = {}, [], True, {}
     while moved:
         moved = False
         for s, q in queues.items():
@@ -97,6 +124,10 @@ def replay(ops, nbytes):
                 op = q[pos[s]]
                 if op[0] == "wait" and done.get(op[2].cuda_event, 0) < op[3]:
                     break
+                if op[0] == "gate" and any(flags.get((op[2], c), 0) < op[3] for c in range(n_flags)):
+                    break
+                if op[0] == "flag":
+                    flags[(op[2], op[3])] = op[4]
                 if op[0] == "record":
                     done[op[2].cuda_event] = max(done.get(op[2].cuda_event, 0), op[3])
                 elif op[0] == "copy":
@@ -111,15 +142,24 @@ def replay(ops, nbytes):
     return seen
 
 
+@pytest.mark.parametrize("gate_slots", [0, 2], ids=["events", "flags"])
 @pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
 @pytest.mark.parametrize("n_layers", [1, 2, 3, 4])
-def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_layers):
+def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_layers, gate_slots):
+    """Event-gated schedule: the compute stream waits for ready.  Flag-gated
+    schedule: the grouped GEMM of execution g waits on the device for every
+    chunk flag of its buffer to reach g + 1; each flag must be written only
+    after its chunk holds the right layer, and never for a later fetch before
+    the grouped GEMM that needs the earlier one has run."""
     monkeypatch.setattr(torch.cuda, "Stream", FakeStream)
     monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
     monkeypatch.setattr(L, "moe_prefetch_layer", fake_prefetch)
+    monkeypatch.setattr(L, "moe_prefetch_layer_flagged", fake_prefetch_flagged)
     monkeypatch.setattr(L, "check", lambda status: None)
     Log.ops = []
-    nbytes = 1000  # an odd size: the halves split at a 256-byte boundary
+    # events: an odd size (the halves split at a 256-byte boundary); flags:
+    # 5 slots of 256 bytes, 2 per flag (3 flags, the last one short)
+    nbytes = 1000 if gate_slots == 0 else 5 * 256
 
     # the constructor's device allocations replaced by pointer stand-ins
     pipe = layer_mod.PrefetchPipeline.__new__(layer_mod.PrefetchPipeline)
@@ -127,6 +167,12 @@ def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_l
     pipe.peer_stores = [Buffer(("store", l)) for l in range(n_layers)]
     pipe.remote_bytes, pipe.chunk_bytes = nbytes, 0
     pipe.split, pipe.pending = split, None
+    pipe.gate_slots, pipe.window_block, pipe.gate_timeout_ns = gate_slots, None, 0
+    n_flags = 0
+    if gate_slots:
+        pipe.stride, n_flags = 256, 3
+        pipe.n_flags = n_flags
+        pipe.flags = [FlagBuffer(("flags", 0), n_flags), FlagBuffer(("flags", 1), n_flags)]
     pipe.bufs = [Buffer(("buf", 0)), Buffer(("buf", 1))]
     pipe.copy_stream = FakeStream(name="copy")
     pipe.ready = [FakeEvent() for _ in range(2)]
@@ -141,7 +187,7 @@ def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_l
     for i in range(n_exec):
         pipe.run_layer(i % n_layers, None, compute, prefetch=True, wrap=True)
 
-    seen = replay(Log.ops, nbytes)
+    seen = replay(Log.ops, nbytes, n_flags)
     assert len(seen) == n_exec
     for i, (lidx, content) in enumerate(seen):
         assert lidx == i % n_layers
@@ -160,6 +206,7 @@ def test_split_halves_cover_the_buffer_once(monkeypatch):
     pipe.peer_stores = [Buffer("store")]
     pipe.bufs = [Buffer("buf0"), Buffer("buf1")]
     pipe.remote_bytes, pipe.chunk_bytes = 16_911_433_728, 0
+    pipe.gate_slots, pipe.g = 0, 0
     pipe.copy_stream = FakeStream(name="copy")
     pipe.ready = [FakeEvent(), FakeEvent()]
     free = FakeEvent()
