@@ -356,6 +356,7 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
     if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.gu_offset, 1,
                                                  lay.bytes, d->H, 2 * d->I, w8)) != MOE_OK)
         return st;
+    a.w_off = lay.gu_offset;
     a.scale_off = lay.gu_scale_offset;
     a.kblocks = d->H / 128;
     if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H, kBoxN)) != MOE_OK) return st;
@@ -375,6 +376,7 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
     if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.down_offset, 1,
                                                  lay.bytes, d->I, d->H, w8)) != MOE_OK)
         return st;
+    a.w_off = lay.down_offset;
     a.scale_off = lay.down_scale_offset;
     a.kblocks = d->I / 128;
     if ((st = encode_act_map(&a.act_map, h, rows, d->I, kBoxN)) != MOE_OK) return st;

@@ -36,6 +36,7 @@ struct alignas(64) FfnArgs {
     // w_base[map] + slot * w_stride[map] + scale_off + 4 * (row_block * kblocks + k_block)
     const uint8_t* w_base[3];
     int64_t w_stride[3];
+    int64_t w_off;           // the matrix (w_gu or w_down) from an image's start
     int64_t scale_off;
     int32_t kblocks;
     // e4m3 activations (tensor-core fp8 path): activation scales [K/128][act_scale_ld]
@@ -149,6 +150,21 @@ __device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G
         run += token_tiles<BN>(tb.n[i]) * MT;
     }
     if (lane == 31) tb.tile_start[G] = incl;
+}
+
+// One look at the readiness flag of a remote slot, without waiting: true if
+// the tile reads no fetch in flight, or its chunk has landed (then ordered
+// like gate_wait).
+__device__ __forceinline__ bool gate_ready(const FfnArgs& p, int map, int slot, int& passed) {
+    if (p.ready_flags == nullptr || map != 1) return true;
+    const int f = slot / p.slots_per_flag;
+    if (f == passed) return true;
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.ready_flags + f) : "memory");
+    if ((int32_t)(v - p.ready_epoch) < 0) return false;
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    passed = f;
+    return true;
 }
 
 // Per-expert readiness of a fetch still in flight: waits until the chunk of
