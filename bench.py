@@ -415,23 +415,36 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
     Restores the pipeline's own schedule afterwards."""
     import torch
     from split_weight_b200 import DenseBlock
+    from split_weight_b200 import _lib as L
     saved = (pipe.split, pipe.gate_slots, pipe.window_block)
     steps = max(3, args.workload_steps)
 
     def run(split, gate_slots, window):
+        """One schedule; a kernel wait that ran out (or another device
+        check) is reported in its entry, not raised."""
         torch.cuda.synchronize()
         pipe.configure(split=split, gate_slots=gate_slots, window_block=window)
         pipe.prime()
         for _ in range(2):
             step()
         torch.cuda.synchronize()
+        st = L.moe_check_device()
+        if st != L.MOE_OK:
+            return {"error": f"{L.status_string(st)} in warm-up: {L.moe_last_error()}"}
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
-        return prefetch_overlap(cfg, pipe, step, stream, e0.elapsed_time(e1) / steps, steps)
+        st = L.moe_check_device()
+        if st != L.MOE_OK:
+            return {"error": f"{L.status_string(st)}: {L.moe_last_error()}"}
+        out = prefetch_overlap(cfg, pipe, step, stream, e0.elapsed_time(e1) / steps, steps)
+        st = L.moe_check_device()
+        if st != L.MOE_OK:
+            out["error"] = f"{L.status_string(st)} in the no-copy or copy-alone runs"
+        return out
 
     out = {"events_halves": run(True, 0, None), "flags_whole": run(False, 8, None),
            "flags_halves": run(True, 8, None)}
@@ -479,7 +492,6 @@ def measure_extra_workload(cfg_id, args, dev, stream, peaks, peak_src):
                                            elapsed_ms / args.workload_steps, args.workload_steps)
         if not args.no_schedules:
             out["prefetch"]["schedules"] = prefetch_schedules(cfg, pipe, step, stream, args, dev)
-        L.check(L.moe_check_device())
     del dls, pipe, step
     gc.collect()
     torch.cuda.synchronize()
@@ -528,7 +540,6 @@ def run_ours(args, rank, world, local_rank):
                                          args.steps)
         if world == 1 and not args.no_schedules:
             prefetch_info["schedules"] = prefetch_schedules(cfg, pipe, step, stream, args, dev)
-        L.check(L.moe_check_device())
 
     # ---- split-weight ablation: merge both pools into one buffer every step
     merge_info = None
@@ -641,7 +652,12 @@ def run_ours(args, rank, world, local_rank):
             w = int(w)
             if w == args.config:
                 continue
-            extra[config(w).name] = measure_extra_workload(w, args, dev, stream, peaks, peak_src)
+            try:
+                extra[config(w).name] = measure_extra_workload(w, args, dev, stream, peaks, peak_src)
+            except Exception as exc:   # an extra measurement never costs the main line
+                extra[config(w).name] = {"error": f"{type(exc).__name__}: {exc}"}
+                gc.collect()
+                torch.cuda.empty_cache()
         out["workloads"] = extra
     return out, cfg
 

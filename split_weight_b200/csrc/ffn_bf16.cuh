@@ -7,20 +7,18 @@
 namespace swb {
 namespace {
 
+constexpr uint32_t kA8Bytes = kBM * kBK;       // one e4m3 weight tile as loaded, 8 KB
 constexpr int kConvThreads = 256;              // e4m3 -> bf16 converter warps (8)
-constexpr int kConvAhead = 3;                  // stages a converter's global loads run ahead
 
-// Per stage: the bf16 weight tile(s) the MMA reads (128-byte swizzled) and
-// the token tile.  e4m3 weights do not pass through shared memory as codes:
-// the converter warps load them from global memory into registers.
+// Per stage: the bf16 weight tile(s) the MMA reads (128-byte swizzled), the
+// token tile, and for e4m3 weights the staging tile(s) TMA writes.
 template <int BN, int MODE, bool W8>
 struct Cfg {
     static constexpr int kNA = MODE == kSingle ? 1 : 2;           // weight tiles per stage
     static constexpr uint32_t kAStage = kABytes * kNA;
     static constexpr uint32_t kBStage = BN * kBK * 2;
-    static constexpr uint32_t kStageBytes = kAStage + kBStage;
-    // 16-byte e4m3 chunks a converter thread loads per stage (64 codes of a row = 4 chunks)
-    static constexpr int kConvLoads = kNA * kBM * (kBK / 16) / kConvThreads;
+    static constexpr uint32_t kA8Stage = W8 ? kA8Bytes * kNA : 0;
+    static constexpr uint32_t kStageBytes = kAStage + kBStage + kA8Stage;
     static constexpr int kStages = (kSmemBudget / kStageBytes) > 12 ? 12 : (kSmemBudget / kStageBytes);
     static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
     static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
@@ -112,7 +110,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
                 if (!gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)) break;
                 const CUtensorMap* wm = &p.w_map[t.map];
-                const uint32_t tx = (W8 ? 0u : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
+                const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
                 const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
                 for (int kb = 0; kb < KB; ++kb) {
                     const uint32_t eb = smem_u32(&empty_bar[stage]);
@@ -123,12 +121,11 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                     }
                     const uint32_t sa = stages + stage * C::kStageBytes;
                     mbar_arrive_expect_tx(fb, tx);
-                    // bf16 weights go straight into the operand tile; e4m3 ones
-                    // are written there by the converter warps
-                    if constexpr (!W8) {
-                        tma_load_3d(sa, wm, fb, kb * kBK, t.m0, t.slot);
-                        if constexpr (C::kNA == 2) tma_load_3d(sa + kABytes, wm, fb, kb * kBK, row_a1, t.slot);
-                    }
+                    // e4m3 weights land in the staging area, bf16 ones straight in the operand
+                    const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
+                    const uint32_t w_step = W8 ? kA8Bytes : kABytes;
+                    tma_load_3d(sw, wm, fb, kb * kBK, t.m0, t.slot);
+                    if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * kBK, row_a1, t.slot);
                     const uint32_t sb = sa + C::kAStage;
                     int r = 0;
                     for (; r + 64 <= t.n_mma; r += 64)
@@ -157,8 +154,8 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
                 const uint32_t idesc = idesc_bf16_f32(kBM, t.n_mma);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err) ||
-                        (W8 && !mbar_wait(smem_u32(&conv_bar[stage]), phase, abort_flag, p.err))) {
+                    const uint32_t ready_bar = W8 ? smem_u32(&conv_bar[stage]) : smem_u32(&full_bar[stage]);
+                    if (!mbar_wait(ready_bar, phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
@@ -187,135 +184,63 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         }
     } else if (W8 && warp >= C::kConvFirstWarp) {
         // ------------------------------------------------ e4m3 -> bf16 converters
-        // Thread ct owns kConvLoads 16-byte chunks of each stage: chunk i is
-        // id = ct + 256 i; weight tile a = id / 512, row r = (id % 512) / 4,
-        // chunk c = id % 4 of the row's 64 codes.  Its codes are loaded from
-        // global memory kConvAhead stages ahead (L2-coherent loads: a gated
-        // fetch may still be writing other slots of the buffer), then, once
-        // the MMA has released the stage, converted with the block scale and
-        // stored in the 128-byte swizzle (16-byte chunk j of row r at
-        // j ^ (r % 8)).  One 128x128 scale block covers a stage.
-        constexpr int kL = C::kConvLoads;
+        // Each staged row is 64 e4m3 bytes (4 chunks of 16); the bf16 operand
+        // row is 128 bytes in the 128-byte swizzle: 16-byte chunk j of row r
+        // sits at position j ^ (r % 8).  One 128x128 block scale covers the
+        // whole stage (64 columns of K, 128 rows).
         const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. kConvThreads-1
-        struct Ahead {
-            uint4 v[kL];
-            float s[2];
-            int tile, kb;      // the stage these codes belong to
-            bool live;         // a stage to convert
-            bool deferred;     // its remote chunk had not landed: load at conversion time
-        };
-        // load cursor: the (tile, kb) whose codes are loaded next
-        int l_tile = blockIdx.x, l_kb = 0, passed = -1, l_map = 0, l_slot = 0;
-        bool l_ready = true;
-        const uint8_t* l_rows[2] = {nullptr, nullptr};   // first code of row block a
-        const float* l_sc[2] = {nullptr, nullptr};      // its block scales
-        auto tile_ptrs = [&](int tile, const uint8_t* (&rows)[2], const float* (&sc)[2], int& map,
-                             int& slot) {
+        int stage = 0, passed = -1;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
-            const uint8_t* img = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map];
-            const int rb1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
-            rows[0] = img + p.w_off + (int64_t)t.m0 * p.K;
-            rows[1] = img + p.w_off + (int64_t)rb1 * p.K;
-            sc[0] = reinterpret_cast<const float*>(img + p.scale_off) + (int64_t)(t.m0 / kBM) * p.kblocks;
-            sc[1] = reinterpret_cast<const float*>(img + p.scale_off) + (int64_t)(rb1 / kBM) * p.kblocks;
-            map = t.map;
-            slot = t.slot;
-        };
-        // codes and scales of stage kb of a tile (L2-coherent loads: a gated
-        // fetch may still be writing other slots of the buffer)
-        auto issue = [&](Ahead& b, const uint8_t* const (&rows)[2], const float* const (&sc)[2], int kb) {
+            // the block scales sit in the remote buffer too: read them only once
+            // landed, with L2-coherent loads (a gated fetch may be writing other slots)
+            if (!__all_sync(0xffffffffu, gate_wait(p, t.map, t.slot, passed, abort_flag, p.err))) break;
+            const uint8_t* sbase = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map] + p.scale_off;
+            const float* sc0 = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
+            const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
+            const float* sc1 = reinterpret_cast<const float*>(sbase) + (int64_t)rb1 * p.kblocks;
+            for (int kb = 0; kb < KB; ++kb) {
+                const float s0 = __ldcg(sc0 + (kb >> 1));
+                const float s1 = C::kNA == 2 ? __ldcg(sc1 + (kb >> 1)) : 0.0f;
+                ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = stages + stage * C::kStageBytes;
+                const uint32_t s8 = sa + C::kAStage + C::kBStage;
 #pragma unroll
-            for (int i = 0; i < kL; ++i) {
-                // tile a = (ct + 256 i) / 512 = i / 2 (ct < 256): known at compile time
-                const int a = (kConvThreads * i) >> 9, r = ((ct + kConvThreads * i) >> 2) & 127, c = ct & 3;
-                const uint8_t* src = (a == 0 ? rows[0] : rows[1]) + (int64_t)r * p.K + kb * kBK + c * 16;
-                asm volatile("ld.global.cg.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(b.v[i].x), "=r"(b.v[i].y), "=r"(b.v[i].z), "=r"(b.v[i].w)
-                             : "l"(src));
-            }
-            b.s[0] = __ldcg(sc[0] + (kb >> 1));
-            b.s[1] = C::kNA == 2 ? __ldcg(sc[1] + (kb >> 1)) : 0.0f;
-        };
-        // The codes and scales of a remote expert sit in the buffer a gated
-        // fetch fills: they are loaded only once its chunk has landed.  The
-        // run-ahead load only looks at the flag; a stage whose chunk is still
-        // in flight is loaded when it is converted, after waiting there, so
-        // that a remote tile never holds up the stages of the tile before it.
-        auto load = [&](Ahead& b) {
-            b.live = l_tile < total;
-            if (!b.live) return;
-            b.tile = l_tile;
-            b.kb = l_kb;
-            if (!l_ready) l_ready = __all_sync(0xffffffffu, gate_ready(p, l_map, l_slot, passed));
-            b.deferred = !l_ready;
-            if (l_ready) issue(b, l_rows, l_sc, l_kb);
-            if (++l_kb == KB) {
-                l_kb = 0;
-                l_tile += gridDim.x;
-                if (l_tile < total) {
-                    tile_ptrs(l_tile, l_rows, l_sc, l_map, l_slot);
-                    l_ready = __all_sync(0xffffffffu, gate_ready(p, l_map, l_slot, passed));
+                for (int a = 0; a < C::kNA; ++a) {
+                    const float sc = a == 0 ? s0 : s1;
+#pragma unroll
+                    for (int i = 0; i < (kBM * kBK / 16) / kConvThreads; ++i) {
+                        const int id = ct + kConvThreads * i, r = id >> 2, c = id & 3;
+                        uint4 in, lo, hi;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(in.x), "=r"(in.y), "=r"(in.z), "=r"(in.w)
+                                     : "r"(s8 + a * kA8Bytes + r * kBK + c * 16));
+                        e4m3x16_to_bf16(in, sc, lo, hi);
+                        const uint32_t row = sa + a * kABytes + r * 128;
+                        const uint32_t j0 = (2 * c) ^ (r & 7), j1 = (2 * c + 1) ^ (r & 7);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j0 * 16),
+                                     "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
+                                     : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j1 * 16),
+                                     "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                                     : "memory");
+                    }
+                }
+                // generic-proxy stores -> visible to the tensor core's async proxy
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&conv_bar[stage]));
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-        };
-        int stage = 0;
-        uint32_t phase = 0;
-        auto convert = [&](Ahead& b) -> bool {   // false: nothing left, or aborted
-            if (!b.live) return false;
-            if (b.deferred) {
-                const uint8_t* rows[2];
-                const float* sc[2];
-                int map, slot;
-                tile_ptrs(b.tile, rows, sc, map, slot);
-                if (!__all_sync(0xffffffffu, gate_wait(p, map, slot, passed, abort_flag, p.err)))
-                    return false;
-                issue(b, rows, sc, b.kb);
-            }
-            // the MMA must have finished reading this stage's previous contents
-            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u,
-                                                   abort_flag, p.err)))
-                return false;
-            const uint32_t sa = stages + stage * C::kStageBytes;
-#pragma unroll
-            for (int i = 0; i < kL; ++i) {
-                const int a = (kConvThreads * i) >> 9, r = ((ct + kConvThreads * i) >> 2) & 127, c = ct & 3;
-                uint4 lo, hi;
-                e4m3x16_to_bf16(b.v[i], a == 0 ? b.s[0] : b.s[1], lo, hi);
-                const uint32_t row = sa + a * kABytes + r * 128;
-                const uint32_t j0 = (2 * c) ^ (r & 7), j1 = (2 * c + 1) ^ (r & 7);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j0 * 16),
-                             "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
-                             : "memory");
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j1 * 16),
-                             "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
-                             : "memory");
-            }
-            // generic-proxy stores -> visible to the tensor core's async proxy
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&conv_bar[stage]));
-            if (++stage == C::kStages) {
-                stage = 0;
-                phase ^= 1u;
-            }
-            return true;
-        };
-        static_assert(kConvAhead == 3, "the loop below is unrolled for three stages in flight");
-        Ahead b0, b1, b2;
-        if (l_tile < total) {
-            tile_ptrs(l_tile, l_rows, l_sc, l_map, l_slot);
-            l_ready = __all_sync(0xffffffffu, gate_ready(p, l_map, l_slot, passed));
-        }
-        load(b0);
-        load(b1);
-        load(b2);
-        while (true) {
-            if (!convert(b0)) break;
-            load(b0);
-            if (!convert(b1)) break;
-            load(b1);
-            if (!convert(b2)) break;
-            load(b2);
         }
     } else {
         // ------------------------------------------------ epilogue

@@ -23,6 +23,7 @@ struct alignas(64) FfnArgs {
     CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}
     CUtensorMap act_map;       // activation rows {K, rows}, 16-row box
     CUtensorMap act_map64;     // the same rows, 64-row box
+    CUtensorMap w_map4[3];     // CTA-pair gate/up kernel: {K, gate|up, feature, slot}, box 64 x 2 x 64
     const int32_t* offsets;    // [E+1] first row of each expert
     __nv_bfloat16* out;        // [rows, ld_out]
     int* err;                  // device error word
@@ -36,7 +37,6 @@ struct alignas(64) FfnArgs {
     // w_base[map] + slot * w_stride[map] + scale_off + 4 * (row_block * kblocks + k_block)
     const uint8_t* w_base[3];
     int64_t w_stride[3];
-    int64_t w_off;           // the matrix (w_gu or w_down) from an image's start
     int64_t scale_off;
     int32_t kblocks;
     // e4m3 activations (tensor-core fp8 path): activation scales [K/128][act_scale_ld]
@@ -78,21 +78,22 @@ struct Tables {
 // An expert's n rows are cut into equal token tiles of tr rows (a multiple of
 // 16, at most BN): tiles of one expert that stream the same weights then run
 // at the same pace, so the second one finds the weights still in L2.
-template <int BN>
+// AL: the MMA row granule of a tile (16; 32 when a CTA pair splits it in halves).
+template <int BN, int AL = 16>
 __device__ __host__ __forceinline__ int tile_rows(int n) {
     const int ntn = (n + BN - 1) / BN;
     const int per = (n + ntn - 1) / ntn;
-    return (per + 15) & ~15;
+    return (per + AL - 1) & ~(AL - 1);
 }
 
-template <int BN>
+template <int BN, int AL = 16>
 __device__ __host__ __forceinline__ int token_tiles(int n) {
     if (n <= 0) return 0;
-    const int tr = tile_rows<BN>(n);
+    const int tr = tile_rows<BN, AL>(n);
     return (n + tr - 1) / tr;
 }
 
-template <int BN, int ROWS>
+template <int BN, int ROWS, int AL = 16>
 __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
     int lo = 0, hi = G - 1;
     while (lo < hi) {  // largest group whose first tile is <= tile (never an empty one)
@@ -101,14 +102,14 @@ __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
         else hi = mid - 1;
     }
     const int g = lo, local = tile - tb.tile_start[g], n = tb.n[g];
-    const int tr = tile_rows<BN>(n);
+    const int tr = tile_rows<BN, AL>(n);
     const int ntn = (n + tr - 1) / tr;
     const int mt = local / ntn, nt = local - mt * ntn;
     Tile t;
     t.m0 = mt * ROWS;
     t.row0 = tb.row0[g] + nt * tr;
     t.n_rows = min(tr, n - nt * tr);
-    t.n_mma = (t.n_rows + 15) & ~15;
+    t.n_mma = (t.n_rows + AL - 1) & ~(AL - 1);
     t.map = tb.ps[g] >> 24;
     t.slot = tb.ps[g] & 0xFFFFFF;
     return t;
@@ -116,7 +117,7 @@ __device__ __forceinline__ Tile decode_tile(int tile, const Tables& tb, int G) {
 
 // One warp: per position (group p.order[i]) the first row, rows, tile count
 // and (pool, slot), and the exclusive scan of tiles over the positions.
-template <int BN>
+template <int BN, int AL = 16>
 __device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G, int MT, int lane) {
     const int per = (G + 31) / 32, i0 = lane * per, i1 = min(G, i0 + per);
     int sum = 0;
@@ -136,7 +137,7 @@ __device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G
         tb.row0[i] = r0;
         tb.n[i] = n;
         tb.ps[i] = ps;
-        sum += token_tiles<BN>(n) * MT;
+        sum += token_tiles<BN, AL>(n) * MT;
     }
     int incl = sum;
 #pragma unroll
@@ -147,7 +148,7 @@ __device__ __forceinline__ void build_tables(const FfnArgs& p, Tables& tb, int G
     int run = incl - sum;
     for (int i = i0; i < i1; ++i) {
         tb.tile_start[i] = run;
-        run += token_tiles<BN>(tb.n[i]) * MT;
+        run += token_tiles<BN, AL>(tb.n[i]) * MT;
     }
     if (lane == 31) tb.tile_start[G] = incl;
 }
@@ -199,7 +200,13 @@ __device__ __forceinline__ bool gate_wait(const FfnArgs& p, int map, int slot, i
     return true;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// silu(g) * u = g / (1 + e^-g) * u with the fast exponential and division
+// (a few ulp in fp32; h is rounded to bf16 or e4m3 right after).  For
+// g < -87, 1 + e^-g exceeds 2^126 and __fdividef gives 0, which is silu(g)
+// rounded to any output format.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
 
 }  // namespace
 }  // namespace swb

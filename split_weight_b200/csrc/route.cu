@@ -171,13 +171,17 @@ __global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
     extern __shared__ float ls[];  // [kBigT][kBigLd]: sum of the finished chunks, per pair
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int e0 = blockIdx.x * kBigE, t0 = blockIdx.y * kBigT;
-    // loader mapping: w  -> expert lt = tid / 2, h offset (tid % 2) * 8   (8 values)
-    //                 x  -> token  lt (threads with lt < 64 only)
-    const int lt = tid >> 1, lh = (tid & 1) * 8;
-    const bool xload = lt < kBigT;
-    const bool xin = xload && t0 + lt < T, win = e0 + lt < E;
-    const XT* xrow = x + (int64_t)(xin ? t0 + lt : 0) * H + lh;
-    const float* wrow = wg + (int64_t)(win ? e0 + lt : 0) * H + lh;
+    // loader mapping, 8 consecutive h per thread:
+    //   w -> expert  tid % 128, h offset (tid / 128) * 8
+    //   x -> token   tid % 64,  h offset (tid / 64) * 8   (threads < 128)
+    // so that the 32 lanes of a warp store 32 consecutive columns of one
+    // stage row (no bank conflicts in store())
+    const int lw = tid & 127, lhw = (tid >> 7) * 8;
+    const int lx = tid & 63, lhx = ((tid >> 6) & 1) * 8;
+    const bool xload = tid < 2 * kBigT;
+    const bool xin = xload && t0 + lx < T, win = e0 + lw < E;
+    const XT* xrow = x + (int64_t)(xin ? t0 + lx : 0) * H + lhx;
+    const float* wrow = wg + (int64_t)(win ? e0 + lw : 0) * H + lhw;
     float rx[8], rw[8];
     auto load = [&](int h0) {
         if constexpr (sizeof(XT) == 2) {
@@ -203,8 +207,8 @@ __global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
     auto store = [&](int buf) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            if (xload) xs[buf][lh + i][lt] = rx[i];
-            ws[buf][lh + i][lt] = rw[i];
+            if (xload) xs[buf][lhx + i][lx] = rx[i];
+            ws[buf][lhw + i][lw] = rw[i];
         }
     };
     auto row_of = [&](int i) { return ty * 4 + i; };

@@ -16,6 +16,7 @@ from oracle import workload as ow
 from split_weight_b200 import _lib as L
 
 from gpu_util import (DECODE_FP8, MAX_EXPERTS, MID_BN128, MID_BN128_FP8, MID_BN256, MID_BN256_FP8,
+                      MID_BN256_H384,
                       MID_FP8, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16, RTOL_FP8,
                       SPARSE_DECODE, assert_close_rel, run_layer, sync_check, to_np)
 
@@ -76,13 +77,14 @@ def test_small_layer_full_parity(cfg):
     assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
 
 
-@pytest.mark.parametrize("cfg", [MID_BN256, MID_BN256_FP8, MID_BN128, MID_BN128_FP8],
+@pytest.mark.parametrize("cfg", [MID_BN256, MID_BN256_H384, MID_BN256_FP8, MID_BN128, MID_BN128_FP8],
                          ids=lambda c: c.name)
 def test_mid_layer_each_tile_width_full_parity(cfg):
     """Whole mid-size layers whose experts get ~256 or ~125 tokens each, so
-    the grouped GEMMs run 256-token tiles (one 512-column TMEM accumulator
-    set, the wide epilogue) or 128-token tiles with ragged row counts;
-    every output element against the oracle."""
+    the grouped GEMMs run 256-token tiles (bf16 weights: CTA pairs with
+    interleaved gate/up rows; e4m3 weights: single CTAs with one 512-column
+    accumulator set) or 128-token tiles with ragged row counts; every output
+    element against the oracle."""
     dl = mdev.build_layer(cfg)
     run_layer(dl)
     y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)

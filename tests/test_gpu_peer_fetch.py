@@ -40,6 +40,7 @@ def test_each_rank_receives_the_other_pools_in_rank_order(cuda_device, slices):
         ready = torch.cuda.Event()
         ready.record(copy)
         peers = PeerPools(G, r, [p.data_ptr() for p in pools], nbytes, slices)
+        copy.wait_stream(torch.cuda.current_stream())   # dst and the pools are filled there
         peers.fetch(dst, copy, None, ready)
         assert L.moe_wait_ready(ready.cuda_event, 20000) == L.MOE_OK
         want = torch.cat([pools[s] for s in range(G) if s != r])
@@ -69,6 +70,7 @@ def test_pool_exported_by_another_process_is_fetched(cuda_device):
         own = _pool(0, nbytes, cuda_device)
         dst = torch.zeros(nbytes, dtype=torch.uint8, device=cuda_device)
         copy = torch.cuda.Stream()
+        copy.wait_stream(torch.cuda.current_stream())   # dst is zero-filled there
         PeerPools(2, 0, [own.data_ptr(), base], nbytes, 4).fetch(dst, copy)
         copy.synchronize()
         assert torch.equal(dst, _pool(1, nbytes, cuda_device))
