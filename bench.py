@@ -48,7 +48,7 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-merge-ablation", action="store_true")
-    p.add_argument("--prefetch-split", type=int, default=1, choices=(0, 1),
+    p.add_argument("--prefetch-split", type=int, default=0, choices=(0, 1),
                    help="issue each layer's fetch in two halves in the windows between grouped GEMMs")
     p.add_argument("--act-dtype", choices=["bf16", "e4m3"], default="bf16",
                    help="activations the grouped GEMMs read (e4m3: opt-in fp8 tensor-core path, "
@@ -56,9 +56,10 @@ def parse_args(argv=None):
     p.add_argument("--workloads", default="3,4,5",
                    help="further workloads measured in the same run (1 GPU only; '' for none)")
     p.add_argument("--workload-steps", type=int, default=5)
-    p.add_argument("--gate-slots", type=int, default=0,
-                   help="pipelined workloads: per-chunk readiness flags every N remote slots "
-                        "instead of waiting for the whole fetch (0: event-gated)")
+    p.add_argument("--gate-slots", type=int, default=8,
+                   help="pipelined workloads: per-chunk readiness flags every N remote slots, "
+                        "the grouped GEMM starting before the fetch ends (0: the compute stream "
+                        "waits for the whole fetch)")
     p.add_argument("--window-inter", type=int, default=12288,
                    help="intermediate size of the dense block that stands in for the attention "
                         "block in the prefetch-window measurement (0: skip it)")

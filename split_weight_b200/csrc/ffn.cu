@@ -27,7 +27,6 @@
 // holds up the next tile's MMA is short.
 #include "ffn_bf16.cuh"
 #include "ffn_f8.cuh"
-#include "ffn_pair.cuh"
 
 namespace swb {
 namespace {
@@ -60,64 +59,6 @@ moe_status launch_bn(int bn, const FfnArgs& a, int rows, int G, cudaStream_t s) 
         case 128: return launch<128, MODE, W8>(a, rows, G, s);
         default: return launch<256, MODE, W8>(a, rows, G, s);
     }
-}
-
-// CTA pairs of the pair kernel that can be resident at once (cached per
-// device): its grid is persistent, so it must not exceed them.
-template <int MODE>
-moe_status pair_capacity(int* out) {
-    using C = CfgPair<MODE>;
-    static int cached[64] = {0};
-    int dev = 0;
-    SWB_CUDA(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device %d", dev);
-    if (!cached[dev]) {
-        auto kern = k_grouped_ffn_pair<MODE>;
-        SWB_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)C::kDynSmem));
-        int sms = 0;
-        moe_status st = sm_count(&sms);
-        if (st != MOE_OK) return st;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-        cfg.blockDim = dim3(C::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = C::kDynSmem;
-        int n = 0;
-        SWB_CUDA(cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kern), &cfg));
-        if (n <= 0) return fail(MOE_ERR_UNSUPPORTED, "no CTA pair of the grouped FFN fits on device %d", dev);
-        cached[dev] = n;
-    }
-    *out = cached[dev];
-    return MOE_OK;
-}
-
-template <int MODE>
-moe_status launch_pair(const FfnArgs& a, int rows, int G, cudaStream_t s) {
-    using C = CfgPair<MODE>;
-    int cap = 0;
-    moe_status st = pair_capacity<MODE>(&cap);
-    if (st != MOE_OK) return st;
-    const int64_t mt = a.M / C::kRowsPerTile;
-    const int64_t bound = mt * ((rows + C::kAL - 1) / C::kAL + G);
-    const int pairs = (int)(bound < cap ? bound : cap);
-    if (pairs <= 0) return MOE_OK;
-    k_grouped_ffn_pair<MODE><<<2 * pairs, C::kThreads, C::kDynSmem, s>>>(a);
-    SWB_LAUNCHED(MODE == kGated ? "moe_grouped_ffn: gate/up kernel (CTA pairs)"
-                                : "moe_grouped_ffn: down kernel (CTA pairs)");
-    return MOE_OK;
-}
-
-// 4-D map {K, gate|up, feature, slot} over one pool's w_gu: a box of 64
-// features x {gate, up} x 64 of K lands as 128 rows with the gate and up
-// rows of each feature adjacent (the pair kernel's gate/up operand).
-moe_status encode_gu_map4(CUtensorMap* m, const void* base, int64_t offset, int32_t count,
-                          int64_t stride, int32_t H, int32_t I) {
-    const uint64_t dims[4] = {(uint64_t)H, 2u, (uint64_t)I, (uint64_t)count};
-    const uint64_t strides[3] = {(uint64_t)I * H * 2, (uint64_t)H * 2, (uint64_t)stride};
-    const uint32_t box[4] = {(uint32_t)kBK, 2u, 64u, 1u};
-    return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                        const_cast<char*>(static_cast<const char*>(base)) + offset, dims, strides,
-                        box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <int BN, int MODE>
@@ -407,27 +348,14 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
     if (f8) return ffn_f8(d, tbl, lay, x_perm, x_perm_scales, h, y_perm,
                           static_cast<float*>(workspace), (int)rows, G, a, stream);
 
-    // 256-token tiles with bf16 weights run on CTA pairs (double-buffered
-    // accumulators); every other shape on single CTAs
-    const bool pairs = bn == 256 && !w8;
     // GEMM1: h = silu(X W_gate^T) * (X W_up^T)
-    if (pairs) {
-        for (int q = 0; q < 2; ++q)
-            if (count[q] > 0 && (st = encode_gu_map4(&a.w_map4[q], base[q], lay.gu_offset, count[q],
-                                                     stride[q], d->H, d->I)) != MOE_OK)
-                return st;
-        if (d->has_shared && (st = encode_gu_map4(&a.w_map4[2], tbl->shared, lay.gu_offset, 1,
-                                                  lay.bytes, d->H, d->I)) != MOE_OK)
+    for (int q = 0; q < 2; ++q)
+        if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.gu_offset, count[q],
+                                                    stride[q], d->H, 2 * d->I, w8)) != MOE_OK)
             return st;
-    } else {
-        for (int q = 0; q < 2; ++q)
-            if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.gu_offset, count[q],
-                                                        stride[q], d->H, 2 * d->I, w8)) != MOE_OK)
-                return st;
-        if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.gu_offset, 1,
-                                                     lay.bytes, d->H, 2 * d->I, w8)) != MOE_OK)
-            return st;
-    }
+    if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.gu_offset, 1,
+                                                 lay.bytes, d->H, 2 * d->I, w8)) != MOE_OK)
+        return st;
     a.scale_off = lay.gu_scale_offset;
     a.kblocks = d->H / 128;
     if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H, kBoxN)) != MOE_OK) return st;
@@ -437,9 +365,7 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
     a.up_row = d->I;
     a.out = static_cast<__nv_bfloat16*>(h);
     a.ld_out = d->I;
-    st = pairs ? launch_pair<kGated>(a, (int)rows, G, stream)
-               : launch_w<kGated>(w8, bn, a, (int)rows, G, stream);
-    if (st != MOE_OK) return st;
+    if ((st = launch_w<kGated>(w8, bn, a, (int)rows, G, stream)) != MOE_OK) return st;
 
     // GEMM2: y = h W_down^T
     for (int q = 0; q < 2; ++q)
@@ -458,9 +384,7 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
     a.up_row = 0;
     a.out = static_cast<__nv_bfloat16*>(y_perm);
     a.ld_out = d->H;
-    if (d->H % (2 * kBM) == 0)
-        return pairs ? launch_pair<kPair>(a, (int)rows, G, stream)
-                     : launch_w<kPair>(w8, bn, a, (int)rows, G, stream);
+    if (d->H % (2 * kBM) == 0) return launch_w<kPair>(w8, bn, a, (int)rows, G, stream);
     return launch_w<kSingle>(w8, bn, a, (int)rows, G, stream);
 }
 

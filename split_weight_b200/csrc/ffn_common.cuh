@@ -23,7 +23,6 @@ struct alignas(64) FfnArgs {
     CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}
     CUtensorMap act_map;       // activation rows {K, rows}, 16-row box
     CUtensorMap act_map64;     // the same rows, 64-row box
-    CUtensorMap w_map4[3];     // CTA-pair gate/up kernel: {K, gate|up, feature, slot}, box 64 x 2 x 64
     const int32_t* offsets;    // [E+1] first row of each expert
     __nv_bfloat16* out;        // [rows, ld_out]
     int* err;                  // device error word

@@ -32,7 +32,7 @@ DECODE_FP8 = config(5).with_(cfg_id=25, name="decode_fp8_T7_H256_I128_E64", T=7,
 MID_BN256 = config(2).with_(cfg_id=27, name="mid_bn256_T2048_H512_I256_E8_k1", T=2048, H=512,
                             I=256, E=8, k=1, n_group=1, topk_group=1, local_count=3)
 # the same with H = 384: the down GEMM's 256-row tiles do not divide H, so it
-# runs 128-row tiles on single CTAs beside the gate/up GEMM on CTA pairs
+# runs single 128-row tiles
 MID_BN256_H384 = config(2).with_(cfg_id=31, name="mid_bn256_T2048_H384_I256_E8_k1", T=2048, H=384,
                                  I=256, E=8, k=1, n_group=1, topk_group=1, local_count=3)
 MID_BN256_FP8 = config(5).with_(cfg_id=28, name="mid_bn256_fp8_T2048_H512_I256_E8_k1", T=2048,

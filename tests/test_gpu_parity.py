@@ -81,10 +81,10 @@ def test_small_layer_full_parity(cfg):
                          ids=lambda c: c.name)
 def test_mid_layer_each_tile_width_full_parity(cfg):
     """Whole mid-size layers whose experts get ~256 or ~125 tokens each, so
-    the grouped GEMMs run 256-token tiles (bf16 weights: CTA pairs with
-    interleaved gate/up rows; e4m3 weights: single CTAs with one 512-column
-    accumulator set) or 128-token tiles with ragged row counts; every output
-    element against the oracle."""
+    the grouped GEMMs run 256-token tiles (one 512-column TMEM accumulator
+    set, the wide epilogue) or 128-token tiles with ragged row counts, in the
+    two-tile (gate/up, paired down) and single-tile (H = 384) down modes;
+    every output element against the oracle."""
     dl = mdev.build_layer(cfg)
     run_layer(dl)
     y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
