@@ -279,7 +279,7 @@ def make_step(cfg, dls, pipe, stream):
             ml.permute(inputs[0], h)
             if timed_ffn is not None:
                 timed_ffn[0][0].record(stream)
-            ml.grouped_ffn(h)
+            ml.grouped_ffn(h, x=inputs[0])
             if timed_ffn is not None:
                 timed_ffn[0][1].record(stream)
             ml.combine(h)
@@ -703,7 +703,7 @@ def merge_ablation(cfg, dl, stream, split_step_ms: float, reps: int):
             merge()
             ml.route(dl.x, h)
             ml.permute(dl.x, h)
-            ml.grouped_ffn(h)
+            ml.grouped_ffn(h, x=dl.x)
             ml.combine(h)
         ev[3].record(stream)
         torch.cuda.synchronize()

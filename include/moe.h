@@ -297,6 +297,21 @@ MOE_API moe_status moe_grouped_ffn_gated(const moe_ffn_desc *d, const moe_expert
                                  void *y_perm, void *workspace, size_t workspace_bytes,
                                  cudaStream_t stream);
 
+/* moe_grouped_ffn_gated with GEMM1's token rows read from x itself instead
+ * of x_perm: the row gather of moe_permute is fused into the GEMM's operand
+ * load (TMA tile::gather4 through perm_src), so x_perm need not be written
+ * (moe_permute with x_perm = NULL).  Routed row r of expert e reads
+ * x[perm_src[r]]; the shared expert's rows are x[0 .. T-1].
+ * x [T, H] bf16 (act_dtype must be MOE_BF16; w_dtype MOE_BF16 or MOE_E4M3);
+ * perm_src [T*k] int32 as moe_permute wrote it, 16-byte aligned.  A perm_src
+ * value outside [0, T) is reported through the device error word
+ * (MOE_ERR_DEVICE_CHECK) and token 0 is read in its place.  gate may be NULL.
+ * Everything else as moe_grouped_ffn. */
+MOE_API moe_status moe_grouped_ffn_x(const moe_ffn_desc *d, const moe_expert_table *tbl,
+                             const moe_ready_gate *gate, const void *x, const int32_t *perm_src,
+                             const int32_t *offsets, void *h, void *y_perm, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Weighted combine (unpermute):
  *   y[t] = sum_{j=0..k-1, ascending} topk_w[t,j] * y_perm[inv_pos[t,j]]

@@ -81,7 +81,7 @@ class DeviceLayer:
 
 
 def build_layer(cfg, layer: int = 0, device="cuda", placement=None,
-                act_dtype: str | None = None) -> DeviceLayer:
+                act_dtype: str | None = None, gather: bool | None = None) -> DeviceLayer:
     from split_weight_b200 import MoELayer, SplitWeights
     cfg = config(cfg)
     li = gen.layer_inputs(cfg, layer)
@@ -90,7 +90,7 @@ def build_layer(cfg, layer: int = 0, device="cuda", placement=None,
     fill_weights(cfg, layer, w)
     wg = torch.from_numpy(li.wg).to(device)
     bias = torch.from_numpy(li.bias).to(device) if li.bias is not None else None
-    ml = MoELayer(layer_shape(cfg, act_dtype), wg, bias, w, device)
+    ml = MoELayer(layer_shape(cfg, act_dtype), wg, bias, w, device, gather=gather)
     return DeviceLayer(cfg, layer, li, x_tensor(li, device), ml, pool, slot)
 
 

@@ -90,6 +90,8 @@ _SIGS = {
     "moe_grouped_ffn_gated": ([ctypes.POINTER(moe_ffn_desc), ctypes.POINTER(moe_expert_table),
                                ctypes.POINTER(moe_ready_gate), vp, vp, vp, vp, vp, vp, sz, vp], i32),
     "moe_prefetch_layer_flagged": ([vp, vp, sz, sz, vp, vp, vp, ctypes.c_uint32, vp], i32),
+    "moe_grouped_ffn_x": ([ctypes.POINTER(moe_ffn_desc), ctypes.POINTER(moe_expert_table),
+                           ctypes.POINTER(moe_ready_gate), vp, vp, vp, vp, vp, vp, sz, vp], i32),
     "moe_combine": ([i32, i32, i32, vp, vp, vp, i32, vp, i32, vp], i32),
     "moe_prefetch_layer": ([vp, vp, sz, sz, vp, vp, vp], i32),
     "moe_peer_fetch_plan": ([i32, i32, i64, i32, ctypes.POINTER(moe_peer_copy), i32,
@@ -140,6 +142,7 @@ moe_expert_layout_get = _lib.moe_expert_layout_get
 moe_grouped_ffn_workspace_size = _lib.moe_grouped_ffn_workspace_size
 moe_grouped_ffn = _lib.moe_grouped_ffn
 moe_grouped_ffn_gated = _lib.moe_grouped_ffn_gated
+moe_grouped_ffn_x = _lib.moe_grouped_ffn_x
 moe_prefetch_layer_flagged = _lib.moe_prefetch_layer_flagged
 moe_combine = _lib.moe_combine
 moe_prefetch_layer = _lib.moe_prefetch_layer

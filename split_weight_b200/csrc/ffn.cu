@@ -235,6 +235,11 @@ moe_status ffn_f8(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_
     return launch_f8_bn<kPair>(bn, a, rows, G, stream);
 }
 
+moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_ready_gate* gate,
+                   const void* x_perm, const float* x_perm_scales, const int32_t* perm_src,
+                   const int32_t* offsets, void* h, void* y_perm, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream);
+
 }  // namespace
 }  // namespace swb
 
@@ -262,6 +267,34 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
                                  const float* x_perm_scales, const int32_t* offsets, void* h,
                                  void* y_perm, void* workspace, size_t workspace_bytes,
                                  cudaStream_t stream) {
+    return ffn_run(d, tbl, gate, x_perm, x_perm_scales, nullptr, offsets, h, y_perm, workspace,
+                   workspace_bytes, stream);
+}
+
+moe_status moe_grouped_ffn_x(const moe_ffn_desc* d, const moe_expert_table* tbl,
+                             const moe_ready_gate* gate, const void* x, const int32_t* perm_src,
+                             const int32_t* offsets, void* h, void* y_perm, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+    if (d && d->act_dtype != MOE_BF16)
+        return fail(MOE_ERR_UNSUPPORTED, "moe_grouped_ffn_x: activations must be bf16 (dtype %d)",
+                    d->act_dtype);
+    if (d && d->T > 0 && (!perm_src || !aligned(perm_src, 16)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_x: perm_src NULL or not 16-byte aligned");
+    return ffn_run(d, tbl, gate, x, nullptr, perm_src, offsets, h, y_perm, workspace,
+                   workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace swb {
+namespace {
+
+// The grouped FFN behind both entry points: the token tiles of GEMM1 come from
+// `act` = x_perm (perm_src NULL) or from `act` = x through perm_src.
+moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_ready_gate* gate,
+                   const void* x_perm, const float* x_perm_scales, const int32_t* perm_src,
+                   const int32_t* offsets, void* h, void* y_perm, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
     moe_expert_layout lay;
     moe_status st = validate(d, tbl, &lay);
     if (st != MOE_OK) return st;
@@ -358,8 +391,19 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
         return st;
     a.scale_off = lay.gu_scale_offset;
     a.kblocks = d->H / 128;
-    if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H, kBoxN)) != MOE_OK) return st;
-    if ((st = encode_act_map(&a.act_map64, x_perm, rows, d->H, 64)) != MOE_OK) return st;
+    if (perm_src) {   // token tiles gathered from x [T, H] through perm_src
+        const uint64_t dims[2] = {(uint64_t)d->H, (uint64_t)d->T};
+        const uint64_t strides[1] = {(uint64_t)d->H * 2};
+        const uint32_t box[2] = {(uint32_t)kBK, 1u};
+        if ((st = encode_tiled(&a.x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x_perm),
+                               dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != MOE_OK)
+            return st;
+        a.perm_src = perm_src;
+        a.gather = 1;
+    } else {
+        if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H, kBoxN)) != MOE_OK) return st;
+        if ((st = encode_act_map(&a.act_map64, x_perm, rows, d->H, 64)) != MOE_OK) return st;
+    }
     a.K = d->H;
     a.M = d->I;
     a.up_row = d->I;
@@ -377,6 +421,7 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
         return st;
     a.scale_off = lay.down_scale_offset;
     a.kblocks = d->I / 128;
+    a.gather = 0;
     if ((st = encode_act_map(&a.act_map, h, rows, d->I, kBoxN)) != MOE_OK) return st;
     if ((st = encode_act_map(&a.act_map64, h, rows, d->I, 64)) != MOE_OK) return st;
     a.K = d->I;
@@ -388,4 +433,5 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
     return launch_w<kSingle>(w8, bn, a, (int)rows, G, stream);
 }
 
-}  // extern "C"
+}  // namespace
+}  // namespace swb

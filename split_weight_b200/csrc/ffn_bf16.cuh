@@ -85,8 +85,12 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
             mbar_init(smem_u32(&acc_empty[a]), C::kEpiWarps);
         }
         fence_mbar_init();
-        tma_prefetch_map(&p.act_map);
-        tma_prefetch_map(&p.act_map64);
+        if (p.gather) {
+            tma_prefetch_map(&p.x_map);
+        } else {
+            tma_prefetch_map(&p.act_map);
+            tma_prefetch_map(&p.act_map64);
+        }
         for (int m = 0; m < 3; ++m) tma_prefetch_map(&p.w_map[m]);
     }
     if (warp == 1) {
@@ -102,40 +106,79 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int stage = 0, passed = -1;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
-                if (!gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)) break;
-                const CUtensorMap* wm = &p.w_map[t.map];
-                const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
-                const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
-                for (int kb = 0; kb < KB; ++kb) {
-                    const uint32_t eb = smem_u32(&empty_bar[stage]);
-                    const uint32_t fb = smem_u32(&full_bar[stage]);
-                    if (!mbar_wait(eb, phase ^ 1u, abort_flag, p.err)) {
-                        ok = false;
-                        break;
+        // Lane 0 arms each stage and loads the weight tile(s).  The token
+        // tile comes from x_perm in 64- and 16-row boxes (lane 0) or, with
+        // p.gather, straight from x through perm_src: four rows per
+        // tile::gather4 load, lane i loading rows 4i..4i+3 and 128+4i..131+4i.
+        // Rows past the tile's tokens repeat its last token (their products
+        // are never stored).
+        int stage = 0, passed = -1;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+            if (!__all_sync(0xffffffffu, lane != 0 || gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)))
+                break;
+            const CUtensorMap* wm = &p.w_map[t.map];
+            const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
+            const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
+            int tok[8];
+            if (p.gather) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = (j >> 2) * 128 + 4 * lane + (j & 3);
+                    const int rr = min(r, t.n_rows - 1);
+                    int v = 0;
+                    if (r < t.n_mma) {
+                        // the shared expert's rows are the tokens in order
+                        v = t.map == 2 ? t.row0 + rr - p.A : __ldg(p.perm_src + t.row0 + rr);
+                        if (v < 0 || v >= p.T) {   // not a token: report, read token 0
+                            atomicOr(p.err, kDevErrIndex);
+                            v = 0;
+                        }
                     }
-                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    tok[j] = v;
+                }
+            }
+            for (int kb = 0; kb < KB; ++kb) {
+                const uint32_t eb = smem_u32(&empty_bar[stage]);
+                const uint32_t fb = smem_u32(&full_bar[stage]);
+                bool w = true;
+                if (lane == 0) w = mbar_wait(eb, phase ^ 1u, abort_flag, p.err);
+                if (!__shfl_sync(0xffffffffu, w, 0)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = stages + stage * C::kStageBytes;
+                const uint32_t sb = sa + C::kAStage;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(fb, tx);
                     // e4m3 weights land in the staging area, bf16 ones straight in the operand
                     const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
                     const uint32_t w_step = W8 ? kA8Bytes : kABytes;
                     tma_load_3d(sw, wm, fb, kb * kBK, t.m0, t.slot);
                     if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * kBK, row_a1, t.slot);
-                    const uint32_t sb = sa + C::kAStage;
-                    int r = 0;
-                    for (; r + 64 <= t.n_mma; r += 64)
-                        tma_load_2d(sb + r * kBK * 2, &p.act_map64, fb, kb * kBK, t.row0 + r);
-                    for (; r < t.n_mma; r += kBoxN)
-                        tma_load_2d(sb + r * kBK * 2, &p.act_map, fb, kb * kBK, t.row0 + r);
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
+                    if (!p.gather) {
+                        int r = 0;
+                        for (; r + 64 <= t.n_mma; r += 64)
+                            tma_load_2d(sb + r * kBK * 2, &p.act_map64, fb, kb * kBK, t.row0 + r);
+                        for (; r < t.n_mma; r += kBoxN)
+                            tma_load_2d(sb + r * kBK * 2, &p.act_map, fb, kb * kBK, t.row0 + r);
                     }
+                }
+                __syncwarp();
+                if (p.gather) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int r0 = h * 128 + 4 * lane;
+                        if (r0 < t.n_mma)
+                            tma_gather4(sb + r0 * kBK * 2, &p.x_map, fb, kb * kBK, tok[4 * h],
+                                        tok[4 * h + 1], tok[4 * h + 2], tok[4 * h + 3]);
+                    }
+                }
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
         }

@@ -23,7 +23,10 @@ struct alignas(64) FfnArgs {
     CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}
     CUtensorMap act_map;       // activation rows {K, rows}, 16-row box
     CUtensorMap act_map64;     // the same rows, 64-row box
+    CUtensorMap x_map;         // gathered token tiles: x [T, K] bf16, 64 x 1 box (tile::gather4)
     const int32_t* offsets;    // [E+1] first row of each expert
+    const int32_t* perm_src;   // [T*k] token of each permuted row (gather != 0)
+    int32_t gather;            // token tiles read from x through perm_src, not from x_perm
     __nv_bfloat16* out;        // [rows, ld_out]
     int* err;                  // device error word
     int32_t E, T, A, has_shared;

@@ -143,13 +143,22 @@ class ReadyGate:
 
 
 class MoELayer:
-    """One MoE layer with preallocated device buffers."""
+    """One MoE layer with preallocated device buffers.
+
+    With gather (the default when x and the GEMM activations are bf16) the
+    grouped GEMM reads its token rows from x through perm_src
+    (moe_grouped_ffn_x) and moe_permute writes no x_perm; otherwise x_perm is
+    gathered first (bf16 from fp32 x, or e4m3 with scales)."""
 
     def __init__(self, shape: LayerShape, w_gate: torch.Tensor, bias: torch.Tensor | None,
-                 weights: SplitWeights, device: torch.device | str = "cuda"):
+                 weights: SplitWeights, device: torch.device | str = "cuda",
+                 gather: bool | None = None):
         s = shape
         self.shape, self.w_gate, self.bias, self.weights = s, w_gate, bias, weights
         dev = torch.device(device)
+        can_gather = s.x_dtype == "bf16" and s.act_dtype == "bf16"
+        self.gather = can_gather if gather is None else gather
+        assert can_gather or not self.gather, "gathered token tiles need bf16 x and activations"
         self._cfg = s.route_cfg()
         self._desc = s.ffn_desc()
         i32 = torch.int32
@@ -165,7 +174,8 @@ class MoELayer:
         rows = max(s.rows, 1)
         a8 = s.act_dtype == "e4m3"
         adt = torch.uint8 if a8 else torch.bfloat16
-        self.x_perm = torch.empty(rows, s.H, dtype=adt, device=dev)
+        # with gather x_perm is never written: a one-row placeholder
+        self.x_perm = torch.empty(1 if self.gather else rows, s.H, dtype=adt, device=dev)
         self.x_scales = torch.empty(s.H // 128, rows, dtype=torch.float32, device=dev) if a8 else None
         self.h = torch.empty(rows, s.I, dtype=adt, device=dev)
         self.ffn_ws = torch.empty(max(L.moe_grouped_ffn_workspace_size(ctypes.byref(self._desc)), 16),
@@ -186,18 +196,28 @@ class MoELayer:
         L.check(L.moe_permute(s.T, s.k, s.E, s.H, self.topk_idx.data_ptr(), x.data_ptr(),
                               _DT[s.x_dtype], _DT[s.act_dtype], 1 if s.has_shared else 0,
                               self.offsets.data_ptr(), self.perm_src.data_ptr(),
-                              self.inv_pos.data_ptr(), self.x_perm.data_ptr(),
+                              self.inv_pos.data_ptr(),
+                              None if self.gather else self.x_perm.data_ptr(),
                               _ptr(self.x_scales),
                               self.perm_ws.data_ptr(), self.perm_ws.numel(), stream))
 
     def grouped_ffn(self, stream: int, remote: torch.Tensor | None = None,
-                    gate: "ReadyGate | None" = None) -> None:
+                    gate: "ReadyGate | None" = None, x: torch.Tensor | None = None) -> None:
         """The grouped GEMMs; with a gate, remote experts are read only once
-        their chunk of a fetch still in flight has landed."""
+        their chunk of a fetch still in flight has landed.  x: the layer
+        input, needed when the token rows are gathered from it."""
         tbl = self.weights.table(remote)
         g = gate.c_struct() if gate is not None else None
-        L.check(L.moe_grouped_ffn_gated(ctypes.byref(self._desc), ctypes.byref(tbl),
-                                        ctypes.byref(g) if g is not None else None,
+        gp = ctypes.byref(g) if g is not None else None
+        if self.gather:
+            assert x is not None, "the gathered grouped GEMM reads the layer input x"
+            L.check(L.moe_grouped_ffn_x(ctypes.byref(self._desc), ctypes.byref(tbl), gp,
+                                        x.data_ptr(), self.perm_src.data_ptr(),
+                                        self.offsets.data_ptr(), self.h.data_ptr(),
+                                        self.y_perm.data_ptr(), self.ffn_ws.data_ptr(),
+                                        self.ffn_ws.numel(), stream))
+            return
+        L.check(L.moe_grouped_ffn_gated(ctypes.byref(self._desc), ctypes.byref(tbl), gp,
                                         self.x_perm.data_ptr(), _ptr(self.x_scales),
                                         self.offsets.data_ptr(), self.h.data_ptr(),
                                         self.y_perm.data_ptr(), self.ffn_ws.data_ptr(),
@@ -215,7 +235,7 @@ class MoELayer:
         h = _stream_handle(stream)
         self.route(x, h)
         self.permute(x, h)
-        self.grouped_ffn(h, remote)
+        self.grouped_ffn(h, remote, x=x)
         self.combine(h)
         return self.y
 
@@ -356,7 +376,7 @@ class PrefetchPipeline:
             stream.wait_event(self.ready[b])
         if ffn_events is not None:
             ffn_events[0].record(stream)
-        layer.grouped_ffn(h, self.bufs[b], gate)
+        layer.grouped_ffn(h, self.bufs[b], gate, x=x)
         if ffn_events is not None:
             ffn_events[1].record(stream)
         if prefetch and self.split:

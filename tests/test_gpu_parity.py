@@ -52,6 +52,8 @@ def _check_permutation(dl, idx_ref):
     np.testing.assert_array_equal(ml.inv_pos[:c.T].cpu().numpy(), inv)
     if ml.shape.act_dtype != "bf16":
         return   # e4m3 rows: see test_e4m3_gather_quantises_each_128_block
+    if ml.gather:
+        return   # no x_perm: the grouped GEMM gathers from x (test_x_perm_path_full_parity)
     # gathered rows: x (rounded to bf16 when it came as fp32), then the shared rows
     xp = ml.x_perm[:c.rows].view(torch.int16).cpu().numpy().view(np.uint16)
     xb = gen.f32_to_bf16_bits(dl.inputs.x)
@@ -95,6 +97,27 @@ def test_mid_layer_each_tile_width_full_parity(cfg):
     assert (mean > 160) if cfg.k == 1 else (32 < mean <= 160), "tile width not reached"
     assert (counts % 16 != 0).any(), "no ragged token tile"
     assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
+
+
+@pytest.mark.parametrize("cfg", [MID_SIGMOID, MID_BN256, MID_BN128_FP8, SPARSE_DECODE],
+                         ids=lambda c: c.name)
+def test_x_perm_path_full_parity(cfg):
+    """The grouped GEMM reading x_perm, the rows moe_permute gathers, instead of
+    gathering them itself from x (the default for bf16 inputs): x_perm bit for
+    bit, every output element against the oracle, and bit-identical outputs
+    between the two paths."""
+    dl = mdev.build_layer(cfg, gather=False)
+    assert not dl.layer.gather
+    run_layer(dl)
+    y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
+    _check_routing(dl, idx_ref, w_ref)
+    _check_permutation(dl, idx_ref)
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y (x_perm)")
+    y_xperm = dl.layer.y.clone()
+    g = mdev.build_layer(cfg, gather=True)
+    assert g.layer.gather
+    run_layer(g)
+    assert torch.equal(g.layer.y, y_xperm)
 
 
 @pytest.mark.parametrize("cfg", [MID_FP8, DECODE_FP8, MID_BN128_FP8], ids=lambda c: c.name)
@@ -193,7 +216,7 @@ def test_out_of_range_expert_index_is_reported(cuda_device):
     here before the call): the gather must check it before reading x, zero
     the row and report it; the combine must see inv_pos = -1 and skip it."""
     cfg = SPARSE_DECODE
-    dl = mdev.build_layer(cfg)
+    dl = mdev.build_layer(cfg, gather=False)
     ml = dl.layer
     h = torch.cuda.current_stream().cuda_stream
     ml.route(dl.x, h)
@@ -210,10 +233,31 @@ def test_out_of_range_expert_index_is_reported(cuda_device):
     assert int(ml.inv_pos[0, 0]) == -1
     assert int(ml.perm_src[cfg.A - 1]) == 2**31 - 1          # never written
     assert not ml.x_perm[cfg.A - 1].any()                      # zero-filled, not read from x
-    ml.grouped_ffn(h)
+    ml.grouped_ffn(h, x=dl.x)
     ml.combine(h)
     torch.cuda.synchronize()
     assert L.moe_check_device() == L.MOE_ERR_DEVICE_CHECK     # the combine saw inv_pos = -1
+    assert torch.isfinite(ml.y[:cfg.T].float()).all()
+
+
+def test_gathered_token_rows_check_perm_src(cuda_device):
+    """The grouped GEMM that gathers its token rows from x through perm_src
+    checks every value against [0, T) before the load: a corrupt entry is
+    reported (MOE_ERR_DEVICE_CHECK) and token 0 read in its place."""
+    cfg = SPARSE_DECODE
+    dl = mdev.build_layer(cfg)
+    ml = dl.layer
+    assert ml.gather
+    h = torch.cuda.current_stream().cuda_stream
+    ml.route(dl.x, h)
+    ml.permute(dl.x, h)
+    torch.cuda.synchronize()
+    ml.perm_src[0] = 2**31 - 1
+    ml.grouped_ffn(h, x=dl.x)
+    ml.combine(h)
+    torch.cuda.synchronize()
+    assert L.moe_check_device() == L.MOE_ERR_DEVICE_CHECK
+    assert L.moe_check_device() == L.MOE_OK
     assert torch.isfinite(ml.y[:cfg.T].float()).all()
 
 

@@ -48,7 +48,7 @@ def test_gate_with_flags_landed_equals_ungated(cfg, act):
     h = torch.cuda.current_stream().cuda_stream
     ml.route(dl.x, h)
     ml.permute(dl.x, h)
-    ml.grouped_ffn(h, None, gate)
+    ml.grouped_ffn(h, None, gate, x=dl.x)
     ml.combine(h)
     sync_check()
     assert torch.equal(ml.y, y_ref)
@@ -101,7 +101,7 @@ def test_flag_never_written_times_out_and_library_stays_usable(cfg, act):
     ml.permute(dl.x, h)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    ml.grouped_ffn(h, None, gate)
+    ml.grouped_ffn(h, None, gate, x=dl.x)
     torch.cuda.synchronize()
     waited = time.perf_counter() - t0
     assert L.moe_check_device() == L.MOE_ERR_TIMEOUT

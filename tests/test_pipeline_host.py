@@ -65,7 +65,7 @@ class FakeLayer:
     def permute(self, x, h):
         pass
 
-    def grouped_ffn(self, h, remote, gate=None):
+    def grouped_ffn(self, h, remote, gate=None, x=None):
         if gate is not None:   # the gated kernel reads each chunk once its flag reached the epoch
             Log.ops.append(("gate", "compute", gate.flags.owner, gate.epoch))
         Log.ops.append(("ffn", "compute", self.idx, remote.owner))
