@@ -171,17 +171,19 @@ __global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
     extern __shared__ float ls[];  // [kBigT][kBigLd]: sum of the finished chunks, per pair
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int e0 = blockIdx.x * kBigE, t0 = blockIdx.y * kBigT;
-    // loader mapping, 8 consecutive h per thread:
-    //   w -> expert  tid % 128, h offset (tid / 128) * 8
-    //   x -> token   tid % 64,  h offset (tid / 64) * 8   (threads < 128)
-    // so that the 32 lanes of a warp store 32 consecutive columns of one
-    // stage row (no bank conflicts in store())
-    const int lw = tid & 127, lhw = (tid >> 7) * 8;
-    const int lx = tid & 63, lhx = ((tid >> 6) & 1) * 8;
-    const bool xload = tid < 2 * kBigT;
-    const bool xin = xload && t0 + lx < T, win = e0 + lw < E;
-    const XT* xrow = x + (int64_t)(xin ? t0 + lx : 0) * H + lhx;
-    const float* wrow = wg + (int64_t)(win ? e0 + lw : 0) * H + lhw;
+    // loader mapping: w  -> expert lt = tid / 2, h offset (tid % 2) * 8   (8 values)
+    //                 x  -> token  lt (threads with lt < 64 only)
+    // Two lanes share a row's 16 h.  Stored in step, their stage rows lh + i
+    // would sit 8 apart, and rows 8 apart hit the same banks at any 16-byte
+    // row stride.  The odd lane stores its values rotated by four: the pair
+    // writes rows i and 8 + (i + 4) % 8, 4 or 12 apart, which at a stride of
+    // 4 banks per row puts its 16 columns on the other 16 banks.
+    const int lt = tid >> 1, lh = (tid & 1) * 8;
+    const bool odd = tid & 1;
+    const bool xload = lt < kBigT;
+    const bool xin = xload && t0 + lt < T, win = e0 + lt < E;
+    const XT* xrow = x + (int64_t)(xin ? t0 + lt : 0) * H + lh;
+    const float* wrow = wg + (int64_t)(win ? e0 + lt : 0) * H + lh;
     float rx[8], rw[8];
     auto load = [&](int h0) {
         if constexpr (sizeof(XT) == 2) {
@@ -207,8 +209,11 @@ __global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
     auto store = [&](int buf) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            if (xload) xs[buf][lhx + i][lx] = rx[i];
-            ws[buf][lhw + i][lw] = rw[i];
+            const int j = odd ? (i + 4) & 7 : i;
+            const float vx = odd ? rx[(i + 4) & 7] : rx[i];
+            const float vw = odd ? rw[(i + 4) & 7] : rw[i];
+            if (xload) xs[buf][lh + j][lt] = vx;
+            ws[buf][lh + j][lt] = vw;
         }
     };
     auto row_of = [&](int i) { return ty * 4 + i; };

@@ -145,10 +145,12 @@ class ReadyGate:
 class MoELayer:
     """One MoE layer with preallocated device buffers.
 
-    With gather (the default when x and the GEMM activations are bf16) the
-    grouped GEMM reads its token rows from x through perm_src
-    (moe_grouped_ffn_x) and moe_permute writes no x_perm; otherwise x_perm is
-    gathered first (bf16 from fp32 x, or e4m3 with scales)."""
+    By default moe_permute gathers x_perm (bf16, from bf16 or fp32 x, or e4m3
+    with scales) and the grouped GEMM reads it.  With gather=True (bf16 x and
+    activations only) the grouped GEMM reads its token rows from x through
+    perm_src instead (moe_grouped_ffn_x) and no x_perm is written; it gives
+    the same bits, and is slower at large batches, where its four-row TMA
+    gathers cannot feed the tensor cores."""
 
     def __init__(self, shape: LayerShape, w_gate: torch.Tensor, bias: torch.Tensor | None,
                  weights: SplitWeights, device: torch.device | str = "cuda",
@@ -157,7 +159,7 @@ class MoELayer:
         self.shape, self.w_gate, self.bias, self.weights = s, w_gate, bias, weights
         dev = torch.device(device)
         can_gather = s.x_dtype == "bf16" and s.act_dtype == "bf16"
-        self.gather = can_gather if gather is None else gather
+        self.gather = bool(gather)
         assert can_gather or not self.gather, "gathered token tiles need bf16 x and activations"
         self._cfg = s.route_cfg()
         self._desc = s.ffn_desc()

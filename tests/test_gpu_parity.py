@@ -53,7 +53,7 @@ def _check_permutation(dl, idx_ref):
     if ml.shape.act_dtype != "bf16":
         return   # e4m3 rows: see test_e4m3_gather_quantises_each_128_block
     if ml.gather:
-        return   # no x_perm: the grouped GEMM gathers from x (test_x_perm_path_full_parity)
+        return   # no x_perm: the grouped GEMM gathers from x (test_gathered_path_full_parity)
     # gathered rows: x (rounded to bf16 when it came as fp32), then the shared rows
     xp = ml.x_perm[:c.rows].view(torch.int16).cpu().numpy().view(np.uint16)
     xb = gen.f32_to_bf16_bits(dl.inputs.x)
@@ -101,23 +101,23 @@ def test_mid_layer_each_tile_width_full_parity(cfg):
 
 @pytest.mark.parametrize("cfg", [MID_SIGMOID, MID_BN256, MID_BN128_FP8, SPARSE_DECODE],
                          ids=lambda c: c.name)
-def test_x_perm_path_full_parity(cfg):
-    """The grouped GEMM reading x_perm, the rows moe_permute gathers, instead of
-    gathering them itself from x (the default for bf16 inputs): x_perm bit for
-    bit, every output element against the oracle, and bit-identical outputs
-    between the two paths."""
-    dl = mdev.build_layer(cfg, gather=False)
-    assert not dl.layer.gather
+def test_gathered_path_full_parity(cfg):
+    """The grouped GEMM gathering its token rows itself from x through
+    perm_src (moe_grouped_ffn_x, TMA tile::gather4) instead of reading the
+    x_perm that moe_permute gathers: every output element against the
+    oracle, and bit-identical to the x_perm path."""
+    dl = mdev.build_layer(cfg, gather=True)
+    assert dl.layer.gather
     run_layer(dl)
     y_ref, idx_ref, w_ref, _ = ow.layer_full(cfg, 0, dl.pool, dl.slot, dl.inputs)
     _check_routing(dl, idx_ref, w_ref)
     _check_permutation(dl, idx_ref)
-    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y (x_perm)")
-    y_xperm = dl.layer.y.clone()
-    g = mdev.build_layer(cfg, gather=True)
-    assert g.layer.gather
-    run_layer(g)
-    assert torch.equal(g.layer.y, y_xperm)
+    assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y (gathered)")
+    y_gathered = dl.layer.y.clone()
+    x = mdev.build_layer(cfg)
+    assert not x.layer.gather
+    run_layer(x)
+    assert torch.equal(x.layer.y, y_gathered)
 
 
 @pytest.mark.parametrize("cfg", [MID_FP8, DECODE_FP8, MID_BN128_FP8], ids=lambda c: c.name)
@@ -197,12 +197,18 @@ def test_kernel_launch_counter(cuda_device):
     """moe_kernel_launches counts each accepted kernel launch: one layer of
     300 tokens is the split router (chunk logits, partial sums, selection),
     permute (histogram, scan, scatter, gather), the two grouped GEMM kernels
-    and the combine; a 0-token layer launches nothing."""
+    and the combine; without the gather kernel when the grouped GEMM gathers
+    its rows itself; a 0-token layer launches nothing."""
     dl = mdev.build_layer(MID_SIGMOID)
     sync_check()
     n0 = L.moe_kernel_launches()
     dl.layer.forward(dl.x)
     assert L.moe_kernel_launches() - n0 == 3 + 4 + 2 + 1
+    dg = mdev.build_layer(MID_SIGMOID, gather=True)
+    sync_check()
+    n0 = L.moe_kernel_launches()
+    dg.layer.forward(dg.x)
+    assert L.moe_kernel_launches() - n0 == 3 + 3 + 2 + 1
     empty = mdev.build_layer(MID_SIGMOID.with_(cfg_id=16, T=0))
     n0 = L.moe_kernel_launches()
     empty.layer.forward(empty.x)
@@ -216,7 +222,7 @@ def test_out_of_range_expert_index_is_reported(cuda_device):
     here before the call): the gather must check it before reading x, zero
     the row and report it; the combine must see inv_pos = -1 and skip it."""
     cfg = SPARSE_DECODE
-    dl = mdev.build_layer(cfg, gather=False)
+    dl = mdev.build_layer(cfg)
     ml = dl.layer
     h = torch.cuda.current_stream().cuda_stream
     ml.route(dl.x, h)
@@ -245,7 +251,7 @@ def test_gathered_token_rows_check_perm_src(cuda_device):
     checks every value against [0, T) before the load: a corrupt entry is
     reported (MOE_ERR_DEVICE_CHECK) and token 0 read in its place."""
     cfg = SPARSE_DECODE
-    dl = mdev.build_layer(cfg)
+    dl = mdev.build_layer(cfg, gather=True)
     ml = dl.layer
     assert ml.gather
     h = torch.cuda.current_stream().cuda_stream
