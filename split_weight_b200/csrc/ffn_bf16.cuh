@@ -7,7 +7,6 @@
 namespace swb {
 namespace {
 
-constexpr uint32_t kA8Bytes = kBM * kBK;       // one e4m3 weight tile as loaded, 8 KB
 constexpr int kConvThreads = 256;              // e4m3 -> bf16 converter warps (8)
 
 // Per stage: the bf16 weight tile(s) the MMA reads (128-byte swizzled), the
@@ -15,9 +14,16 @@ constexpr int kConvThreads = 256;              // e4m3 -> bf16 converter warps (
 template <int BN, int MODE, bool W8>
 struct Cfg {
     static constexpr int kNA = MODE == kSingle ? 1 : 2;           // weight tiles per stage
-    static constexpr uint32_t kAStage = kABytes * kNA;
-    static constexpr uint32_t kBStage = BN * kBK * 2;
-    static constexpr uint32_t kA8Stage = W8 ? kA8Bytes * kNA : 0;
+    // K per stage: 64 (128-byte rows, 128-byte swizzle); 32 (64-byte rows,
+    // 64-byte swizzle) for e4m3 weights at 256-token tiles, where a 64-wide
+    // stage with its e4m3 staging would leave room for two stages only
+    static constexpr int kBKs = (W8 && BN >= 256) ? 32 : kBK;
+    static constexpr bool kSw64 = kBKs == 32;
+    static constexpr uint32_t kATile = kBM * kBKs * 2;            // one bf16 weight tile
+    static constexpr uint32_t kA8Tile = kBM * kBKs;               // one e4m3 tile as loaded
+    static constexpr uint32_t kAStage = kATile * kNA;
+    static constexpr uint32_t kBStage = BN * kBKs * 2;
+    static constexpr uint32_t kA8Stage = W8 ? kA8Tile * kNA : 0;
     static constexpr uint32_t kStageBytes = kAStage + kBStage + kA8Stage;
     static constexpr int kStages = (kSmemBudget / kStageBytes) > 12 ? 12 : (kSmemBudget / kStageBytes);
     static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
@@ -70,7 +76,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     const uint32_t stages = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     const int G = p.E + (p.has_shared ? 1 : 0);
     const int MT = p.M / C::kRowsPerTile;
-    const int KB = p.K / kBK;
+    const int KB = p.K / C::kBKs;
     volatile int* abort_flag = &abort_sh;
 
     if (threadIdx.x == 0) {
@@ -104,11 +110,49 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     const uint32_t tmem_base = tmem_base_sh;
     const int total = tb.tile_start[G];
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        // Lane 0 arms each stage and loads the weight tile(s).  The token
-        // tile comes from x_perm in 64- and 16-row boxes (lane 0) or, with
-        // p.gather, straight from x through perm_src: four rows per
+    if (warp == 0 && !p.gather) {
+        // ------------------------------------------------ TMA producer (one thread)
+        // weight tile(s) and the token tile from x_perm in 64- and 16-row boxes
+        if (lane == 0) {
+            int stage = 0, passed = -1;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
+                if (!gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)) break;
+                const CUtensorMap* wm = &p.w_map[t.map];
+                const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * C::kBKs * 2;
+                const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
+                for (int kb = 0; kb < KB; ++kb) {
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = stages + stage * C::kStageBytes;
+                    mbar_arrive_expect_tx(fb, tx);
+                    // e4m3 weights land in the staging area, bf16 ones straight in the operand
+                    const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
+                    const uint32_t w_step = W8 ? C::kA8Tile : C::kATile;
+                    tma_load_3d(sw, wm, fb, kb * C::kBKs, t.m0, t.slot);
+                    if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * C::kBKs, row_a1, t.slot);
+                    const uint32_t sb = sa + C::kAStage;
+                    int r = 0;
+                    for (; r + 64 <= t.n_mma; r += 64)
+                        tma_load_2d(sb + r * C::kBKs * 2, &p.act_map64, fb, kb * C::kBKs, t.row0 + r);
+                    for (; r < t.n_mma; r += kBoxN)
+                        tma_load_2d(sb + r * C::kBKs * 2, &p.act_map, fb, kb * C::kBKs, t.row0 + r);
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 0) {
+        // ------------------------------------------------ TMA producer (gathered token rows)
+        // Lane 0 arms each stage and loads the weight tile(s); the token tile
+        // comes straight from x through perm_src: four rows per
         // tile::gather4 load, lane i loading rows 4i..4i+3 and 128+4i..131+4i.
         // Rows past the tile's tokens repeat its last token (their products
         // are never stored).
@@ -120,25 +164,23 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
             if (!__all_sync(0xffffffffu, lane != 0 || gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)))
                 break;
             const CUtensorMap* wm = &p.w_map[t.map];
-            const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * kBK * 2;
+            const uint32_t tx = (W8 ? C::kA8Stage : C::kAStage) + (uint32_t)t.n_mma * C::kBKs * 2;
             const int row_a1 = MODE == kGated ? p.up_row + t.m0 : t.m0 + kBM;
             int tok[8];
-            if (p.gather) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = (j >> 2) * 128 + 4 * lane + (j & 3);
-                    const int rr = min(r, t.n_rows - 1);
-                    int v = 0;
-                    if (r < t.n_mma) {
-                        // the shared expert's rows are the tokens in order
-                        v = t.map == 2 ? t.row0 + rr - p.A : __ldg(p.perm_src + t.row0 + rr);
-                        if (v < 0 || v >= p.T) {   // not a token: report, read token 0
-                            atomicOr(p.err, kDevErrIndex);
-                            v = 0;
-                        }
+            for (int j = 0; j < 8; ++j) {
+                const int r = (j >> 2) * 128 + 4 * lane + (j & 3);
+                const int rr = min(r, t.n_rows - 1);
+                int v = 0;
+                if (r < t.n_mma) {
+                    // the shared expert's rows are the tokens in order
+                    v = t.map == 2 ? t.row0 + rr - p.A : __ldg(p.perm_src + t.row0 + rr);
+                    if (v < 0 || v >= p.T) {   // not a token: report, read token 0
+                        atomicOr(p.err, kDevErrIndex);
+                        v = 0;
                     }
-                    tok[j] = v;
                 }
+                tok[j] = v;
             }
             for (int kb = 0; kb < KB; ++kb) {
                 const uint32_t eb = smem_u32(&empty_bar[stage]);
@@ -153,28 +195,18 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 const uint32_t sb = sa + C::kAStage;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(fb, tx);
-                    // e4m3 weights land in the staging area, bf16 ones straight in the operand
                     const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
-                    const uint32_t w_step = W8 ? kA8Bytes : kABytes;
-                    tma_load_3d(sw, wm, fb, kb * kBK, t.m0, t.slot);
-                    if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * kBK, row_a1, t.slot);
-                    if (!p.gather) {
-                        int r = 0;
-                        for (; r + 64 <= t.n_mma; r += 64)
-                            tma_load_2d(sb + r * kBK * 2, &p.act_map64, fb, kb * kBK, t.row0 + r);
-                        for (; r < t.n_mma; r += kBoxN)
-                            tma_load_2d(sb + r * kBK * 2, &p.act_map, fb, kb * kBK, t.row0 + r);
-                    }
+                    const uint32_t w_step = W8 ? C::kA8Tile : C::kATile;
+                    tma_load_3d(sw, wm, fb, kb * C::kBKs, t.m0, t.slot);
+                    if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * C::kBKs, row_a1, t.slot);
                 }
                 __syncwarp();
-                if (p.gather) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int r0 = h * 128 + 4 * lane;
-                        if (r0 < t.n_mma)
-                            tma_gather4(sb + r0 * kBK * 2, &p.x_map, fb, kb * kBK, tok[4 * h],
-                                        tok[4 * h + 1], tok[4 * h + 2], tok[4 * h + 3]);
-                    }
+                for (int h = 0; h < 2; ++h) {
+                    const int r0 = h * 128 + 4 * lane;
+                    if (r0 < t.n_mma)
+                        tma_gather4(sb + r0 * C::kBKs * 2, &p.x_map, fb, kb * C::kBKs, tok[4 * h],
+                                    tok[4 * h + 1], tok[4 * h + 2], tok[4 * h + 3]);
                 }
                 if (++stage == C::kStages) {
                     stage = 0;
@@ -206,12 +238,13 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                     const uint32_t sa = stages + stage * C::kStageBytes;
                     const uint32_t sb = sa + C::kAStage;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                    for (int kk = 0; kk < C::kBKs / 16; ++kk) {
                         const uint32_t accum = (kb | kk) != 0;
-                        const uint64_t bd = sw128_desc(sb + kk * 32);
-                        mma_bf16_ss(d0, sw128_desc(sa + kk * 32), bd, idesc, accum);
+                        const uint64_t bd = C::kSw64 ? sw64_desc(sb + kk * 32) : sw128_desc(sb + kk * 32);
+                        const uint32_t a0 = sa + kk * 32, a1 = a0 + C::kATile;
+                        mma_bf16_ss(d0, C::kSw64 ? sw64_desc(a0) : sw128_desc(a0), bd, idesc, accum);
                         if constexpr (C::kNA == 2)
-                            mma_bf16_ss(d0 + BN, sw128_desc(sa + kABytes + kk * 32), bd, idesc, accum);
+                            mma_bf16_ss(d0 + BN, C::kSw64 ? sw64_desc(a1) : sw128_desc(a1), bd, idesc, accum);
                     }
                     mma_commit(smem_u32(&empty_bar[stage]));
                     if (++stage == C::kStages) {
@@ -227,10 +260,9 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         }
     } else if (W8 && warp >= C::kConvFirstWarp) {
         // ------------------------------------------------ e4m3 -> bf16 converters
-        // Each staged row is 64 e4m3 bytes (4 chunks of 16); the bf16 operand
-        // row is 128 bytes in the 128-byte swizzle: 16-byte chunk j of row r
-        // sits at position j ^ (r % 8).  One 128x128 block scale covers the
-        // whole stage (64 columns of K, 128 rows).
+        // Each staged row is kBKs e4m3 bytes (chunks of 16); the bf16 operand
+        // row is 2 kBKs bytes in the matching swizzle.  One 128x128 block scale
+        // covers the whole stage (kBKs columns of K, 128 rows).
         const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. kConvThreads-1
         int stage = 0, passed = -1;
         uint32_t phase = 0;
@@ -238,15 +270,17 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
             // the block scales sit in the remote buffer too: read them only once
-            // landed, with L2-coherent loads (a gated fetch may be writing other slots)
+            // landed, and L2-coherently while a gated fetch may be writing other slots
             if (!__all_sync(0xffffffffu, gate_wait(p, t.map, t.slot, passed, abort_flag, p.err))) break;
             const uint8_t* sbase = p.w_base[t.map] + (int64_t)t.slot * p.w_stride[t.map] + p.scale_off;
             const float* sc0 = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
             const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
             const float* sc1 = reinterpret_cast<const float*>(sbase) + (int64_t)rb1 * p.kblocks;
             for (int kb = 0; kb < KB; ++kb) {
-                const float s0 = __ldcg(sc0 + (kb >> 1));
-                const float s1 = C::kNA == 2 ? __ldcg(sc1 + (kb >> 1)) : 0.0f;
+                const int sblk = (kb * C::kBKs) >> 7;   // the 128-wide K block of the stage
+                // L1-cached loads, unless a gated fetch may still be writing the buffer
+                const float s0 = p.ready_flags ? __ldcg(sc0 + sblk) : __ldg(sc0 + sblk);
+                const float s1 = C::kNA == 2 ? (p.ready_flags ? __ldcg(sc1 + sblk) : __ldg(sc1 + sblk)) : 0.0f;
                 ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
@@ -258,15 +292,19 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 for (int a = 0; a < C::kNA; ++a) {
                     const float sc = a == 0 ? s0 : s1;
 #pragma unroll
-                    for (int i = 0; i < (kBM * kBK / 16) / kConvThreads; ++i) {
-                        const int id = ct + kConvThreads * i, r = id >> 2, c = id & 3;
+                    for (int i = 0; i < (kBM * C::kBKs / 16) / kConvThreads; ++i) {
+                        constexpr int kCh = C::kBKs / 16;   // 16-code chunks of a staged row
+                        const int id = ct + kConvThreads * i, r = id / kCh, c = id % kCh;
                         uint4 in, lo, hi;
                         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                                      : "=r"(in.x), "=r"(in.y), "=r"(in.z), "=r"(in.w)
-                                     : "r"(s8 + a * kA8Bytes + r * kBK + c * 16));
+                                     : "r"(s8 + a * C::kA8Tile + r * C::kBKs + c * 16));
                         e4m3x16_to_bf16(in, sc, lo, hi);
-                        const uint32_t row = sa + a * kABytes + r * 128;
-                        const uint32_t j0 = (2 * c) ^ (r & 7), j1 = (2 * c + 1) ^ (r & 7);
+                        // the operand row r (kBKs * 2 bytes): 16-byte chunk j at
+                        // j ^ (r % 8) (128-byte swizzle) or j ^ ((r / 2) % 4) (64-byte)
+                        const uint32_t row = sa + a * C::kATile + r * (C::kBKs * 2);
+                        const uint32_t sw = C::kSw64 ? ((r >> 1) & 3) : (r & 7);
+                        const uint32_t j0 = (2 * c) ^ sw, j1 = (2 * c + 1) ^ sw;
                         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j0 * 16),
                                      "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
                                      : "memory");

@@ -206,7 +206,8 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
             for (int j = 0; j < kC; ++j) acc0[j] = acc1[j] = 0.0f;
             float sx[kSx], sxn[kSx];
             load_sx(0, sx);
-            float sw0 = __ldcg(sw0p), sw1 = __ldcg(sw1p);
+            const bool gated = p.ready_flags != nullptr;   // a fetch may still be writing the buffer
+            float sw0 = gated ? __ldcg(sw0p) : __ldg(sw0p), sw1 = gated ? __ldcg(sw1p) : __ldg(sw1p);
             for (int kb = 0; kb < KB; ++kb) {
 #pragma unroll
                 for (int i = 0; i < kSx; ++i) {
@@ -219,8 +220,8 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
                 float sw0n = 0.0f, sw1n = 0.0f;
                 if (kb + 1 < KB) {   // next block's scales travel while this one is folded in
                     load_sx(kb + 1, sxn);
-                    sw0n = __ldcg(sw0p + kb + 1);
-                    sw1n = __ldcg(sw1p + kb + 1);
+                    sw0n = gated ? __ldcg(sw0p + kb + 1) : __ldg(sw0p + kb + 1);
+                    sw1n = gated ? __ldcg(sw1p + kb + 1) : __ldg(sw1p + kb + 1);
                 }
                 ok = mbar_wait(smem_u32(&part_full[pb]), use[pb] & 1u, abort_flag, p.err);
                 if (!__all_sync(0xffffffffu, ok)) {
