@@ -365,17 +365,22 @@ def time_steps(step, cfg, steps, stream, barrier, local_rank, sample_clocks=True
 
 def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
     """Exposed copy time per layer: the same steps without copies, and the
-    copy of one layer's remote experts alone."""
+    copy of one layer's remote experts alone.  Also returns, under
+    "_ffn_ms_no_copy", the grouped FFN's time per step in the steps without
+    copies (the kernels alone, for the roofline)."""
     import torch
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     reps = max(3, min(steps, 10))
+    ffn_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(cfg.layers)] for _ in range(reps)]
     e0.record(stream)
-    for _ in range(reps):
-        step(prefetch=False)
+    for i in range(reps):
+        step(ffn_ev[i], prefetch=False)
     e1.record(stream)
     torch.cuda.synchronize()
     nocopy_ms = e0.elapsed_time(e1) / reps
+    ffn_nocopy = sum(a.elapsed_time(b) for st in ffn_ev for a, b in st) / reps
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     c0.record(pipe.copy_stream)
     pipe.prefetch(0, 0, None)
@@ -398,6 +403,7 @@ def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
         "step_ms_no_copy": round(nocopy_ms, 4),
         "exposed_copy_ms_per_layer": round(exposed, 4),
         "hidden_fraction": round(1.0 - exposed / copy_ms, 4) if copy_ms > 0 else None,
+        "_ffn_ms_no_copy": ffn_nocopy,
     }
 
 
@@ -442,6 +448,7 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
         if st != L.MOE_OK:
             return {"error": f"{L.status_string(st)}: {L.moe_last_error()}"}
         out = prefetch_overlap(cfg, pipe, step, stream, e0.elapsed_time(e1) / steps, steps)
+        out.pop("_ffn_ms_no_copy", None)
         st = L.moe_check_device()
         if st != L.MOE_OK:
             out["error"] = f"{L.status_string(st)} in the no-copy or copy-alone runs"
@@ -461,6 +468,21 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
     pipe.prime()
     torch.cuda.synchronize()
     return out
+
+
+def pipelined_roofline(out, cfg, counts, act, ffn_ms_piped, timed_s, peaks, peak_src):
+    """For a pipelined workload the grouped FFN's time in the pipelined steps
+    includes waiting for chunks of a fetch in flight (readiness flags) and
+    the copy's contention; the roofline takes the kernels alone, from the
+    steps without copies, and keeps the pipelined figure beside it."""
+    pre = out["prefetch"]
+    ffn_alone = pre.pop("_ffn_ms_no_copy")
+    roof = roofline_object(cfg, counts, act, ffn_alone, timed_s, peaks, peak_src)
+    piped = roofline_object(cfg, counts, act, ffn_ms_piped, timed_s, peaks, peak_src)
+    roof["kernel_timing"] = "grouped FFN in the steps without copies (the kernels alone)"
+    roof["frac_with_fetch_in_flight"] = piped["frac"]
+    roof["kernel_ms_per_step_with_fetch"] = piped["kernel_ms_per_step"]
+    out["roofline"] = roof
 
 
 def measure_extra_workload(cfg_id, args, dev, stream, peaks, peak_src):
@@ -491,6 +513,7 @@ def measure_extra_workload(cfg_id, args, dev, stream, peaks, peak_src):
     if pipe is not None:
         out["prefetch"] = prefetch_overlap(cfg, pipe, step, stream,
                                            elapsed_ms / args.workload_steps, args.workload_steps)
+        pipelined_roofline(out, cfg, counts, act, ffn_ms, elapsed_ms / 1e3, peaks, peak_src)
         if not args.no_schedules:
             out["prefetch"]["schedules"] = prefetch_schedules(cfg, pipe, step, stream, args, dev)
     del dls, pipe, step
@@ -539,6 +562,7 @@ def run_ours(args, rank, world, local_rank):
     if pipe is not None:
         prefetch_info = prefetch_overlap(cfg, pipe, step, stream, elapsed_ms / args.steps,
                                          args.steps)
+        ffn_alone_ms = prefetch_info.pop("_ffn_ms_no_copy")
         if world == 1 and not args.no_schedules:
             prefetch_info["schedules"] = prefetch_schedules(cfg, pipe, step, stream, args, dev)
 
@@ -620,6 +644,10 @@ def run_ours(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     roof = roofline_object(cfg, counts, act_dtype, ffn_ms, elapsed_ms / 1e3, peaks, peak_src)
+    if prefetch_info is not None:
+        holder = {"prefetch": dict(prefetch_info, _ffn_ms_no_copy=ffn_alone_ms)}
+        pipelined_roofline(holder, cfg, counts, act_dtype, ffn_ms, elapsed_ms / 1e3, peaks, peak_src)
+        roof = holder["roofline"]
     workload = cfg.name
     nbytes = roof["algorithmic_bytes"]
     out = {
