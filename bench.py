@@ -60,6 +60,11 @@ def parse_args(argv=None):
                    help="pipelined workloads: per-chunk readiness flags every N remote slots, "
                         "the grouped GEMM starting before the fetch ends (0: the compute stream "
                         "waits for the whole fetch)")
+    p.add_argument("--pace-steps", type=int, default=0,
+                   help="pipelined workloads with readiness flags: pace each fetch by the "
+                        "previous grouped GEMM call's progress in N steps (0: unpaced)")
+    p.add_argument("--pace-lead", type=int, default=2,
+                   help="paced fetch: chunks issued before the first progress report")
     p.add_argument("--window-inter", type=int, default=12288,
                    help="intermediate size of the dense block that stands in for the attention "
                         "block in the prefetch-window measurement (0: skip it)")
@@ -258,7 +263,9 @@ def build_workload(cfg, args, dev, act_dtype):
         stores = [mdev.peer_store(cfg, l, dls[l].layer.weights, dev) for l in range(cfg.layers)]
         rbytes = dls[0].layer.weights.n_remote * dls[0].layer.weights.stride
         pipe = PrefetchPipeline([d.layer for d in dls], stores, rbytes, dev,
-                                split=bool(args.prefetch_split), gate_slots=args.gate_slots)
+                                split=bool(args.prefetch_split), gate_slots=args.gate_slots,
+                                pace_steps=args.pace_steps if args.gate_slots > 0 else 0,
+                                pace_lead=args.pace_lead)
         for d in dls:  # the layers' own remote pools are not needed: the buffers replace them
             d.layer.weights.remote = torch.empty(1, dtype=torch.uint8, device=dev)
         torch.cuda.empty_cache()
@@ -393,7 +400,9 @@ def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
     torch.cuda.synchronize()
     exposed = max(0.0, (piped_ms - nocopy_ms) / cfg.layers)
     return {
-        "schedule": (("halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM")
+        "schedule": ((f"paced by the grouped GEMM's progress ({pipe.pace_steps} steps, "
+                      f"{pipe.pace_lead} chunks ahead)" if pipe.pace_steps else
+                      "halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM")
                      + (f"; readiness flags every {pipe.gate_slots} slots" if pipe.gate_slots else
                         "; compute waits for the whole fetch")
                      + ("; dense window block" if pipe.window_block is not None else "")),
@@ -415,7 +424,10 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
                       8 remote slots on the device (readiness flags); the
                       fetch is issued whole as soon as its buffer is free
       flags_halves    the same with the fetch in halves
-      window_*        the same two schedules with a dense compute block
+      flags_paced     flags, the fetch of the next execution issued before
+                      each grouped GEMM call and paced by its progress
+                      reports (24 steps, 2 chunks ahead)
+      window_*        the same schedules with a dense compute block
                       (R1 attention FLOPs) before every MoE block, the
                       explainer's two-block window; its no-copy baseline runs
                       the block too
@@ -423,14 +435,15 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
     import torch
     from split_weight_b200 import DenseBlock
     from split_weight_b200 import _lib as L
-    saved = (pipe.split, pipe.gate_slots, pipe.window_block)
+    saved = (pipe.split, pipe.gate_slots, pipe.window_block, pipe.pace_steps, pipe.pace_lead)
     steps = max(3, args.workload_steps)
 
-    def run(split, gate_slots, window):
+    def run(split, gate_slots, window, pace_steps=0, pace_lead=2):
         """One schedule; a kernel wait that ran out (or another device
         check) is reported in its entry, not raised."""
         torch.cuda.synchronize()
-        pipe.configure(split=split, gate_slots=gate_slots, window_block=window)
+        pipe.configure(split=split, gate_slots=gate_slots, window_block=window,
+                       pace_steps=pace_steps, pace_lead=pace_lead)
         pipe.prime()
         for _ in range(2):
             step()
@@ -455,16 +468,18 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
         return out
 
     out = {"events_halves": run(True, 0, None), "flags_whole": run(False, 8, None),
-           "flags_halves": run(True, 8, None)}
+           "flags_halves": run(True, 8, None), "flags_paced": run(False, 8, None, 24, 2)}
     if args.window_inter > 0:
         block = DenseBlock(cfg.T, cfg.H, args.window_inter, dev)
         out["window_block"] = {"inter": args.window_inter,
                                "flop_per_token": 6.0 * cfg.H * args.window_inter}
         out["window_events_halves"] = run(True, 0, block)
         out["window_flags_whole"] = run(False, 8, block)
+        out["window_flags_paced"] = run(False, 8, block, 24, 2)
         del block
     torch.cuda.synchronize()
-    pipe.configure(split=saved[0], gate_slots=saved[1], window_block=saved[2])
+    pipe.configure(split=saved[0], gate_slots=saved[1], window_block=saved[2],
+                   pace_steps=saved[3], pace_lead=saved[4])
     pipe.prime()
     torch.cuda.synchronize()
     return out

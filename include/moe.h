@@ -312,6 +312,40 @@ MOE_API moe_status moe_grouped_ffn_x(const moe_ffn_desc *d, const moe_expert_tab
                              const int32_t *offsets, void *h, void *y_perm, void *workspace,
                              size_t workspace_bytes, cudaStream_t stream);
 
+/* Progress reports of a grouped-GEMM call, by which a later fetch is paced
+ * (moe_prefetch_layer_paced): the explainer's prefetch caption has the fetch
+ * run while the rank computes; reporting lets the copy spread over that
+ * compute instead of running as one burst beside it.
+ *   word   device, 4-byte aligned: written only by these reports and read by
+ *          the copy stream.  Over one call it takes base + 1 .. base + steps
+ *          as the tiles' MMAs are issued (the gate/up launch covers the first
+ *          round(2 steps / 3) steps, the down launch the rest, each in equal
+ *          parts of its tiles; a wrap-around maximum, never lowered), then
+ *          base + steps + 1 once the call's launches have ended on `stream`,
+ *          finished or stopped early.  A caller that runs calls back to back
+ *          gives call n the base b0 + n (steps + 1).
+ *   tiles  device, two 4-byte words of scratch (tile counters of the two
+ *          launches), reset by the call.
+ *   steps  >= 2. */
+typedef struct moe_progress {
+    uint32_t *word;
+    uint32_t *tiles;
+    uint32_t base;
+    int32_t steps;
+} moe_progress;
+
+/* moe_grouped_ffn_x / moe_grouped_ffn_gated with progress reports.  Token
+ * rows come from x through perm_src when both are given (as in
+ * moe_grouped_ffn_x, x_perm ignored), else from x_perm; gate may be NULL,
+ * progress must not be.  The final write of the progress word is issued
+ * even when the call fails after its argument checks. */
+MOE_API moe_status moe_grouped_ffn_paced(const moe_ffn_desc *d, const moe_expert_table *tbl,
+                                 const moe_ready_gate *gate, const moe_progress *progress,
+                                 const void *x_perm, const float *x_perm_scales, const void *x,
+                                 const int32_t *perm_src, const int32_t *offsets, void *h,
+                                 void *y_perm, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Weighted combine (unpermute):
  *   y[t] = sum_{j=0..k-1, ascending} topk_w[t,j] * y_perm[inv_pos[t,j]]
@@ -423,6 +457,31 @@ MOE_API moe_status moe_prefetch_layer_flagged(const void *src, void *dst, size_t
                                       size_t chunk_bytes, cudaStream_t copy_stream,
                                       cudaEvent_t wait_free, uint32_t *flags, uint32_t epoch,
                                       cudaEvent_t ready_out);
+
+/* moe_prefetch_layer_flagged paced by a grouped-GEMM call's progress (see
+ * moe_progress): before chunk c of n the copy stream waits until
+ *   (int32_t)(*pace->word - moe_pace_threshold(c, n, lead_chunks, pace->base,
+ *                                              pace->steps)) >= 0
+ * (cuStreamWaitValue32, no SM involved).  The first lead_chunks chunks go at
+ * once; the others are spread evenly over the call's reports, the last one
+ * released by report base + steps.  The pacing call must be enqueued on its
+ * stream (or already have run) when the copy stream gets there, or the copy
+ * stream waits for it: issue the fetch and the call together.  Only the
+ * word is read (pace->tiles unused).  MOE_ERR_UNSUPPORTED if the driver
+ * lacks cuStreamWaitValue32 or cuStreamWriteValue32. */
+MOE_API moe_status moe_prefetch_layer_paced(const void *src, void *dst, size_t bytes,
+                                    size_t chunk_bytes, cudaStream_t copy_stream,
+                                    cudaEvent_t wait_free, uint32_t *flags, uint32_t epoch,
+                                    const moe_progress *pace, int32_t lead_chunks,
+                                    cudaEvent_t ready_out);
+
+/* The release threshold of moe_prefetch_layer_paced's chunk c of n:
+ *   c <  lead_chunks:  base
+ *   c >= lead_chunks:  base + floor((c - lead_chunks + 1) (steps + 1)
+ *                                   / (n - lead_chunks + 1))
+ * Host function (no device work). */
+MOE_API uint32_t moe_pace_threshold(int64_t chunk, int64_t n_chunks, int32_t lead_chunks,
+                                    uint32_t base, int32_t steps);
 
 /* Host-side poll of an event with a deadline: MOE_OK once it has completed,
  * MOE_ERR_TIMEOUT after timeout_ms milliseconds, MOE_ERR_CUDA on error. */

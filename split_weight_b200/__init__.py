@@ -9,5 +9,5 @@ pipeline of layers with torch buffers and streams.
 """
 from . import _lib  # noqa: F401  (raises ImportError when the library is missing)
 from ._lib import MoEError, check  # noqa: F401
-from .layer import (DenseBlock, LayerShape, MoELayer, PeerPools, PrefetchPipeline,  # noqa: F401
+from .layer import (DenseBlock, LayerShape, MoELayer, PeerPools, PrefetchPipeline, Progress,  # noqa: F401
                     ReadyGate, SplitWeights, close_pool, export_pool, import_pool)

@@ -60,6 +60,10 @@ class moe_ready_gate(ctypes.Structure):
                 ("n_flags", i32), ("timeout_ns", i64)]
 
 
+class moe_progress(ctypes.Structure):
+    _fields_ = [("word", vp), ("tiles", vp), ("base", ctypes.c_uint32), ("steps", i32)]
+
+
 class MoEError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"{status_string(status)}: {msg}")
@@ -92,6 +96,12 @@ _SIGS = {
     "moe_prefetch_layer_flagged": ([vp, vp, sz, sz, vp, vp, vp, ctypes.c_uint32, vp], i32),
     "moe_grouped_ffn_x": ([ctypes.POINTER(moe_ffn_desc), ctypes.POINTER(moe_expert_table),
                            ctypes.POINTER(moe_ready_gate), vp, vp, vp, vp, vp, vp, sz, vp], i32),
+    "moe_grouped_ffn_paced": ([ctypes.POINTER(moe_ffn_desc), ctypes.POINTER(moe_expert_table),
+                               ctypes.POINTER(moe_ready_gate), ctypes.POINTER(moe_progress), vp,
+                               vp, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+    "moe_prefetch_layer_paced": ([vp, vp, sz, sz, vp, vp, vp, ctypes.c_uint32,
+                                  ctypes.POINTER(moe_progress), i32, vp], i32),
+    "moe_pace_threshold": ([i64, i64, i32, ctypes.c_uint32, i32], ctypes.c_uint32),
     "moe_combine": ([i32, i32, i32, vp, vp, vp, i32, vp, i32, vp], i32),
     "moe_prefetch_layer": ([vp, vp, sz, sz, vp, vp, vp], i32),
     "moe_peer_fetch_plan": ([i32, i32, i64, i32, ctypes.POINTER(moe_peer_copy), i32,
@@ -144,6 +154,9 @@ moe_grouped_ffn = _lib.moe_grouped_ffn
 moe_grouped_ffn_gated = _lib.moe_grouped_ffn_gated
 moe_grouped_ffn_x = _lib.moe_grouped_ffn_x
 moe_prefetch_layer_flagged = _lib.moe_prefetch_layer_flagged
+moe_grouped_ffn_paced = _lib.moe_grouped_ffn_paced
+moe_prefetch_layer_paced = _lib.moe_prefetch_layer_paced
+moe_pace_threshold = _lib.moe_pace_threshold
 moe_combine = _lib.moe_combine
 moe_prefetch_layer = _lib.moe_prefetch_layer
 moe_peer_fetch_plan = _lib.moe_peer_fetch_plan

@@ -111,26 +111,78 @@ moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t ra
     return MOE_OK;
 }
 
-using StreamWriteValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+using StreamValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
 namespace {
-StreamWriteValue32Fn g_write32 = nullptr;
-}
+StreamValue32Fn g_write32 = nullptr, g_wait32 = nullptr;
 
-// cuStreamWriteValue32 through the runtime's driver entry point (the 32-bit
-// stream memory operations of the CUDA 12 driver API need no device opt-in).
-moe_status stream_write_value32(StreamWriteValue32Fn* out) {
+moe_status stream_value_fn(const char* name, StreamValue32Fn* cache, StreamValue32Fn* out) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_write32) {
+    if (!*cache) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cuda_injected_failure())
             return fail(MOE_ERR_CUDA, "cudaGetDriverEntryPoint: injected failure");
-        const cudaError_t e = cudaGetDriverEntryPoint("cuStreamWriteValue32", &fn, cudaEnableDefault, &q);
+        const cudaError_t e = cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q);
         if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
-            return fail(MOE_ERR_UNSUPPORTED, "cuStreamWriteValue32 entry point unavailable");
-        g_write32 = reinterpret_cast<StreamWriteValue32Fn>(fn);
+            return fail(MOE_ERR_UNSUPPORTED, "%s entry point unavailable", name);
+        *cache = reinterpret_cast<StreamValue32Fn>(fn);
     }
-    *out = g_write32;
+    *out = *cache;
+    return MOE_OK;
+}
+}  // namespace
+
+moe_status stream_write_u32(cudaStream_t s, uint32_t* addr, uint32_t value) {
+    StreamValue32Fn fn = nullptr;
+    moe_status st = stream_value_fn("cuStreamWriteValue32", &g_write32, &fn);
+    if (st != MOE_OK) return st;
+    if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "cuStreamWriteValue32: injected failure");
+    const CUresult r = fn(reinterpret_cast<CUstream>(s), reinterpret_cast<CUdeviceptr>(addr), value,
+                          CU_STREAM_WRITE_VALUE_DEFAULT);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuStreamWriteValue32 failed (CUresult %d)", (int)r);
+    return MOE_OK;
+}
+
+moe_status stream_wait_geq_u32(cudaStream_t s, const uint32_t* addr, uint32_t value) {
+    StreamValue32Fn fn = nullptr;
+    moe_status st = stream_value_fn("cuStreamWaitValue32", &g_wait32, &fn);
+    if (st != MOE_OK) return st;
+    if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "cuStreamWaitValue32: injected failure");
+    const CUresult r = fn(reinterpret_cast<CUstream>(s), reinterpret_cast<CUdeviceptr>(addr), value,
+                          CU_STREAM_WAIT_VALUE_GEQ);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuStreamWaitValue32 failed (CUresult %d)", (int)r);
+    return MOE_OK;
+}
+
+uint32_t pace_threshold(int64_t chunk, int64_t n_chunks, int32_t lead_chunks, uint32_t base,
+                        int32_t steps) {
+    if (chunk < lead_chunks) return base;
+    const int64_t paced = n_chunks - lead_chunks, j = chunk - lead_chunks;
+    return base + (uint32_t)(((j + 1) * ((int64_t)steps + 1)) / (paced + 1));
+}
+
+// The chunked copy of moe_prefetch_layer_flagged / _paced: per chunk an
+// optional wait for the progress word, the copy, then the chunk's flag.
+moe_status flagged_copy(const void* src, void* dst, size_t bytes, size_t chunk_bytes,
+                        cudaStream_t copy_stream, cudaEvent_t wait_free, uint32_t* flags,
+                        uint32_t epoch, const moe_progress* pace, int32_t lead_chunks,
+                        cudaEvent_t ready_out) {
+    if (wait_free) SWB_CUDA(cudaStreamWaitEvent(copy_stream, wait_free, 0));
+    const int64_t n = (int64_t)((bytes + chunk_bytes - 1) / chunk_bytes);
+    int64_t c = 0;
+    for (size_t off = 0; off < bytes; off += chunk_bytes, ++c) {
+        moe_status st;
+        if (pace && (st = stream_wait_geq_u32(copy_stream, pace->word,
+                                              pace_threshold(c, n, lead_chunks, pace->base,
+                                                             pace->steps))) != MOE_OK)
+            return st;
+        const size_t len = bytes - off < chunk_bytes ? bytes - off : chunk_bytes;
+        SWB_CUDA(cudaMemcpyAsync(static_cast<char*>(dst) + off,
+                                 static_cast<const char*>(src) + off, len,
+                                 cudaMemcpyDeviceToDevice, copy_stream));
+        if ((st = stream_write_u32(copy_stream, flags + c, epoch)) != MOE_OK) return st;
+    }
+    if (ready_out) SWB_CUDA(cudaEventRecord(ready_out, copy_stream));
     return MOE_OK;
 }
 
@@ -227,25 +279,36 @@ moe_status moe_prefetch_layer_flagged(const void* src, void* dst, size_t bytes, 
             return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_flagged: source and destination "
                         "overlap");
     }
-    StreamWriteValue32Fn write32 = nullptr;
-    moe_status st = stream_write_value32(&write32);
-    if (st != MOE_OK) return st;
-    if (wait_free) SWB_CUDA(cudaStreamWaitEvent(copy_stream, wait_free, 0));
-    size_t c = 0;
-    for (size_t off = 0; off < bytes; off += chunk_bytes, ++c) {
-        const size_t n = bytes - off < chunk_bytes ? bytes - off : chunk_bytes;
-        SWB_CUDA(cudaMemcpyAsync(static_cast<char*>(dst) + off,
-                                 static_cast<const char*>(src) + off, n,
-                                 cudaMemcpyDeviceToDevice, copy_stream));
-        if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "cuStreamWriteValue32: injected failure");
-        const CUresult r = write32(reinterpret_cast<CUstream>(copy_stream),
-                                   reinterpret_cast<CUdeviceptr>(flags + c), epoch,
-                                   CU_STREAM_WRITE_VALUE_DEFAULT);
-        if (r != CUDA_SUCCESS)
-            return fail(MOE_ERR_CUDA, "cuStreamWriteValue32 failed (CUresult %d)", (int)r);
+    return flagged_copy(src, dst, bytes, chunk_bytes, copy_stream, wait_free, flags, epoch, nullptr,
+                        0, ready_out);
+}
+
+moe_status moe_prefetch_layer_paced(const void* src, void* dst, size_t bytes, size_t chunk_bytes,
+                                    cudaStream_t copy_stream, cudaEvent_t wait_free, uint32_t* flags,
+                                    uint32_t epoch, const moe_progress* pace, int32_t lead_chunks,
+                                    cudaEvent_t ready_out) {
+    if (bytes > 0 && (!src || !dst))
+        return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_paced: NULL buffer");
+    if (chunk_bytes == 0 || !flags || !aligned(flags, 4))
+        return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_paced: chunk_bytes > 0 and "
+                    "4-byte aligned flags needed");
+    if (!pace || !pace->word || !aligned(pace->word, 4) || pace->steps < 1 || lead_chunks < 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_paced: a progress word (4-byte "
+                    "aligned), steps >= 1 and lead_chunks >= 0 needed");
+    if (bytes > 0) {
+        const char* s = static_cast<const char*>(src);
+        char* d = static_cast<char*>(dst);
+        if ((s < d + bytes) && (d < s + bytes))
+            return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_layer_paced: source and destination "
+                        "overlap");
     }
-    if (ready_out) SWB_CUDA(cudaEventRecord(ready_out, copy_stream));
-    return MOE_OK;
+    return flagged_copy(src, dst, bytes, chunk_bytes, copy_stream, wait_free, flags, epoch, pace,
+                        lead_chunks, ready_out);
+}
+
+uint32_t moe_pace_threshold(int64_t chunk, int64_t n_chunks, int32_t lead_chunks, uint32_t base,
+                            int32_t steps) {
+    return swb::pace_threshold(chunk, n_chunks, lead_chunks, base, steps);
 }
 
 moe_status moe_wait_ready(cudaEvent_t ev, int32_t timeout_ms) {

@@ -104,10 +104,10 @@ int pick_bn(int64_t A, int E) {
 }
 
 // 3-D map {K, rows, slot} over one pool of expert images.  bf16 weights are
-// loaded straight into the MMA operand layout (128-byte swizzle); e4m3
-// weights as plain 64-byte rows for the converter warps.
-// The e4m3 map for the tensor-core fp8 path (f8mma) loads 128-byte rows
-// straight into the MMA operand layout.
+// loaded straight into the MMA operand layout (bks = 64: 128-byte rows and
+// swizzle; bks = 32: 64-byte rows and swizzle); e4m3 weights as plain
+// bks-byte rows for the converter warps.  The e4m3 map for the tensor-core
+// fp8 path (f8mma) loads 128-byte rows straight into the MMA operand layout.
 moe_status encode_weight_map(CUtensorMap* m, const void* base, int64_t offset, int32_t count,
                              int64_t stride, int32_t K, int32_t rows, bool w8, bool f8mma = false,
                              int bks = kBK) {
@@ -116,7 +116,9 @@ moe_status encode_weight_map(CUtensorMap* m, const void* base, int64_t offset, i
     const uint32_t box[3] = {(uint32_t)(f8mma ? 128 : bks), (uint32_t)kBM, 1u};
     return encode_tiled(m, w8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                         const_cast<char*>(static_cast<const char*>(base)) + offset, dims, strides,
-                        box, (w8 && !f8mma) ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+                        box, (w8 && !f8mma) ? CU_TENSOR_MAP_SWIZZLE_NONE
+                             : (!f8mma && bks == 32) ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                     : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 moe_status encode_act_map8(CUtensorMap* m, const void* base, int64_t rows, int32_t K,
@@ -182,9 +184,24 @@ moe_status validate(const moe_ffn_desc* d, const moe_expert_table* tb, moe_exper
 
 // Both GEMMs on the e4m3 tensor-core path: x_perm and h are e4m3 with
 // per-(row, 128 columns) scales stored [K/128][rows].
+// Progress fields of launch `which` (0 gate/up, 1 down) of a call that
+// reports to `pr` (NULL: none): the gate/up launch covers steps
+// 1 .. round(2 steps / 3), about its share of the FLOPs, the down launch the rest.
+void set_progress(FfnArgs& a, const moe_progress* pr, int which) {
+    if (!pr) {
+        a.progress_word = nullptr;
+        return;
+    }
+    const int s1 = (2 * pr->steps + 1) / 3;
+    a.progress_word = pr->word;
+    a.progress_tiles = pr->tiles + which;
+    a.progress_base = pr->base + (which ? (uint32_t)s1 : 0u);
+    a.progress_steps = which ? pr->steps - s1 : s1;
+}
+
 moe_status ffn_f8(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_expert_layout& lay,
                   const void* x_perm, const float* x_scales, void* h, void* y_perm, float* h_scales,
-                  int rows, int G, FfnArgs& a, cudaStream_t stream) {
+                  int rows, int G, FfnArgs& a, const moe_progress* progress, cudaStream_t stream) {
     moe_status st;
     const void* base[2] = {tbl->local_base, tbl->remote_base};
     const int32_t count[2] = {tbl->local_count, tbl->remote_count};
@@ -213,6 +230,7 @@ moe_status ffn_f8(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_
     a.act_scale_ld = rows;
     a.out8 = static_cast<uint8_t*>(h);
     a.out_scale = h_scales;
+    set_progress(a, progress, 0);
     if ((st = launch_f8_bn<kGated>(bn, a, rows, G, stream)) != MOE_OK) return st;
     // GEMM2 -> y_perm (bf16)
     for (int q = 0; q < 2; ++q)
@@ -234,13 +252,14 @@ moe_status ffn_f8(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_
     a.out = static_cast<__nv_bfloat16*>(y_perm);
     a.out8 = nullptr;
     a.out_scale = nullptr;
+    set_progress(a, progress, 1);
     return launch_f8_bn<kPair>(bn, a, rows, G, stream);
 }
 
 moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_ready_gate* gate,
-                   const void* x_perm, const float* x_perm_scales, const int32_t* perm_src,
-                   const int32_t* offsets, void* h, void* y_perm, void* workspace,
-                   size_t workspace_bytes, cudaStream_t stream);
+                   const moe_progress* progress, const void* x_perm, const float* x_perm_scales,
+                   const int32_t* perm_src, const int32_t* offsets, void* h, void* y_perm,
+                   void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 }  // namespace
 }  // namespace swb
@@ -269,8 +288,8 @@ moe_status moe_grouped_ffn_gated(const moe_ffn_desc* d, const moe_expert_table* 
                                  const float* x_perm_scales, const int32_t* offsets, void* h,
                                  void* y_perm, void* workspace, size_t workspace_bytes,
                                  cudaStream_t stream) {
-    return ffn_run(d, tbl, gate, x_perm, x_perm_scales, nullptr, offsets, h, y_perm, workspace,
-                   workspace_bytes, stream);
+    return ffn_run(d, tbl, gate, nullptr, x_perm, x_perm_scales, nullptr, offsets, h, y_perm,
+                   workspace, workspace_bytes, stream);
 }
 
 moe_status moe_grouped_ffn_x(const moe_ffn_desc* d, const moe_expert_table* tbl,
@@ -282,8 +301,35 @@ moe_status moe_grouped_ffn_x(const moe_ffn_desc* d, const moe_expert_table* tbl,
                     d->act_dtype);
     if (d && d->T > 0 && (!perm_src || !aligned(perm_src, 16)))
         return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_x: perm_src NULL or not 16-byte aligned");
-    return ffn_run(d, tbl, gate, x, nullptr, perm_src, offsets, h, y_perm, workspace,
+    return ffn_run(d, tbl, gate, nullptr, x, nullptr, perm_src, offsets, h, y_perm, workspace,
                    workspace_bytes, stream);
+}
+
+moe_status moe_grouped_ffn_paced(const moe_ffn_desc* d, const moe_expert_table* tbl,
+                                 const moe_ready_gate* gate, const moe_progress* progress,
+                                 const void* x_perm, const float* x_perm_scales, const void* x,
+                                 const int32_t* perm_src, const int32_t* offsets, void* h,
+                                 void* y_perm, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+    if (!progress || !progress->word || !progress->tiles || !aligned(progress->word, 4) ||
+        !aligned(progress->tiles, 4) || progress->steps < 2)
+        return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_paced: progress needs word and tiles "
+                    "(4-byte aligned) and steps >= 2");
+    const bool gather = x && perm_src;
+    moe_status st;
+    if (gather && d && d->act_dtype != MOE_BF16)
+        st = fail(MOE_ERR_UNSUPPORTED, "moe_grouped_ffn_paced: gathered rows need bf16 "
+                  "activations (dtype %d)", d->act_dtype);
+    else if (gather && d && d->T > 0 && !aligned(perm_src, 16))
+        st = fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_paced: perm_src not 16-byte aligned");
+    else
+        st = ffn_run(d, tbl, gate, progress, gather ? x : x_perm, x_perm_scales,
+                     gather ? perm_src : nullptr, offsets, h, y_perm, workspace, workspace_bytes,
+                     stream);
+    // the call's end, done or not: releases every chunk paced by it
+    const moe_status fin = stream_write_u32(stream, progress->word,
+                                            progress->base + (uint32_t)progress->steps + 1u);
+    return st != MOE_OK ? st : fin;
 }
 
 }  // extern "C"
@@ -294,9 +340,9 @@ namespace {
 // The grouped FFN behind both entry points: the token tiles of GEMM1 come from
 // `act` = x_perm (perm_src NULL) or from `act` = x through perm_src.
 moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe_ready_gate* gate,
-                   const void* x_perm, const float* x_perm_scales, const int32_t* perm_src,
-                   const int32_t* offsets, void* h, void* y_perm, void* workspace,
-                   size_t workspace_bytes, cudaStream_t stream) {
+                   const moe_progress* progress, const void* x_perm, const float* x_perm_scales,
+                   const int32_t* perm_src, const int32_t* offsets, void* h, void* y_perm,
+                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     moe_expert_layout lay;
     moe_status st = validate(d, tbl, &lay);
     if (st != MOE_OK) return st;
@@ -374,15 +420,20 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     const int64_t stride[2] = {tbl->local_stride, tbl->remote_stride};
     const int bn = pick_bn(A, d->E);
     const bool w8 = d->w_dtype == MOE_E4M3;
-    const int bks = (w8 && bn >= 256) ? 32 : kBK;   // K per stage of the kernel launched (Cfg::kBKs)
+    const int bks = stage_k(bn, w8);   // K per stage of the kernel launched (Cfg::kBKs)
     a.w_base[0] = static_cast<const uint8_t*>(tbl->local_base);
     a.w_base[1] = static_cast<const uint8_t*>(tbl->remote_base);
     a.w_base[2] = static_cast<const uint8_t*>(tbl->shared);
     a.w_stride[0] = tbl->local_stride;
     a.w_stride[1] = tbl->remote_stride;
     a.w_stride[2] = lay.bytes;
+    if (progress) {   // fresh tile counters for the two launches
+        if ((st = stream_write_u32(stream, progress->tiles, 0u)) != MOE_OK ||
+            (st = stream_write_u32(stream, progress->tiles + 1, 0u)) != MOE_OK)
+            return st;
+    }
     if (f8) return ffn_f8(d, tbl, lay, x_perm, x_perm_scales, h, y_perm,
-                          static_cast<float*>(workspace), (int)rows, G, a, stream);
+                          static_cast<float*>(workspace), (int)rows, G, a, progress, stream);
 
     // GEMM1: h = silu(X W_gate^T) * (X W_up^T)
     for (int q = 0; q < 2; ++q)
@@ -413,6 +464,7 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     a.up_row = d->I;
     a.out = static_cast<__nv_bfloat16*>(h);
     a.ld_out = d->I;
+    set_progress(a, progress, 0);
     if ((st = launch_w<kGated>(w8, bn, a, (int)rows, G, stream)) != MOE_OK) return st;
 
     // GEMM2: y = h W_down^T
@@ -433,6 +485,7 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     a.up_row = 0;
     a.out = static_cast<__nv_bfloat16*>(y_perm);
     a.ld_out = d->H;
+    set_progress(a, progress, 1);
     if (d->H % (2 * kBM) == 0) return launch_w<kPair>(w8, bn, a, (int)rows, G, stream);
     return launch_w<kSingle>(w8, bn, a, (int)rows, G, stream);
 }

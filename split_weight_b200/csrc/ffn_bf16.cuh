@@ -14,10 +14,7 @@ constexpr int kConvThreads = 256;              // e4m3 -> bf16 converter warps (
 template <int BN, int MODE, bool W8>
 struct Cfg {
     static constexpr int kNA = MODE == kSingle ? 1 : 2;           // weight tiles per stage
-    // K per stage: 64 (128-byte rows, 128-byte swizzle); 32 (64-byte rows,
-    // 64-byte swizzle) for e4m3 weights at 256-token tiles, where a 64-wide
-    // stage with its e4m3 staging would leave room for two stages only
-    static constexpr int kBKs = (W8 && BN >= 256) ? 32 : kBK;
+    static constexpr int kBKs = stage_k(BN, W8);                  // K per stage
     static constexpr bool kSw64 = kBKs == 32;
     static constexpr uint32_t kATile = kBM * kBKs * 2;            // one bf16 weight tile
     static constexpr uint32_t kA8Tile = kBM * kBKs;               // one e4m3 tile as loaded
@@ -254,6 +251,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 }
                 if (!ok) break;
                 mma_commit(smem_u32(&acc_full[acc]));
+                report_progress(p, total);
                 ++acc_use[acc];
                 if (C::kAccBufs == 2) acc ^= 1;
             }
@@ -276,11 +274,20 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
             const float* sc0 = reinterpret_cast<const float*>(sbase) + (int64_t)(t.m0 / kBM) * p.kblocks;
             const int rb1 = MODE == kGated ? (p.up_row + t.m0) / kBM : t.m0 / kBM + 1;
             const float* sc1 = reinterpret_cast<const float*>(sbase) + (int64_t)rb1 * p.kblocks;
+            // the block scale of the stage's 128-wide K block: L1-cached loads,
+            // unless a gated fetch may still be writing the buffer
+            auto scale = [&](const float* sc, int kb) {
+                const int sblk = (kb * C::kBKs) >> 7;
+                return p.ready_flags ? __ldcg(sc + sblk) : __ldg(sc + sblk);
+            };
+            // loaded one stage ahead, so that converting a stage never waits on them
+            float s0n = scale(sc0, 0), s1n = C::kNA == 2 ? scale(sc1, 0) : 0.0f;
             for (int kb = 0; kb < KB; ++kb) {
-                const int sblk = (kb * C::kBKs) >> 7;   // the 128-wide K block of the stage
-                // L1-cached loads, unless a gated fetch may still be writing the buffer
-                const float s0 = p.ready_flags ? __ldcg(sc0 + sblk) : __ldg(sc0 + sblk);
-                const float s1 = C::kNA == 2 ? (p.ready_flags ? __ldcg(sc1 + sblk) : __ldg(sc1 + sblk)) : 0.0f;
+                const float s0 = s0n, s1 = s1n;
+                if (kb + 1 < KB) {
+                    s0n = scale(sc0, kb + 1);
+                    if constexpr (C::kNA == 2) s1n = scale(sc1, kb + 1);
+                }
                 ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
@@ -339,35 +346,87 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
             const int f = t.m0 + 32 * q + lane;
             __nv_bfloat16* out = p.out + (int64_t)t.row0 * p.ld_out + f;
             const int c_begin = part * kCols, c_end = min(t.n_rows, c_begin + kCols);
-            for (int c0 = c_begin; c0 < c_end; c0 += 16) {
-                float g[16];
-                tmem_ld_16(tacc + c0, g);
-                if constexpr (C::kNA == 2) {
-                    float u[16];
-                    tmem_ld_16(tacc + BN + c0, u);
-                    tmem_ld_wait();
+            constexpr int kChunks = kCols / 16;
+            constexpr int kOut = (C::kNA == 2 && MODE != kGated) ? 2 : 1;
+            if constexpr (C::kAccBufs == 1 && !W8) {
+                // One accumulator set: the next tile's MMAs wait for it.  Pull this
+                // warp's columns out of TMEM into packed bf16 registers (at most 64),
+                // free the accumulator, then store while the MMAs run.
+                uint32_t pk[kChunks][kOut][8];
+#pragma unroll
+                for (int ch = 0; ch < kChunks; ++ch) {
+                    const int c0 = c_begin + 16 * ch;
+                    if (c0 >= c_end) break;   // warp-uniform
+                    float g[16];
+                    tmem_ld_16(tacc + c0, g);
+                    if constexpr (C::kNA == 2) {
+                        float u[16];
+                        tmem_ld_16(tacc + BN + c0, u);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            if constexpr (MODE == kGated) {
+                                pk[ch][0][i] = pack_bf16x2(silu_mul(g[2 * i], u[2 * i]),
+                                                           silu_mul(g[2 * i + 1], u[2 * i + 1]));
+                            } else {
+                                pk[ch][0][i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+                                pk[ch][kOut - 1][i] = pack_bf16x2(u[2 * i], u[2 * i + 1]);
+                            }
+                        }
+                    } else {
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) pk[ch][0][i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+                uint16_t* out16 = reinterpret_cast<uint16_t*>(out);
+#pragma unroll
+                for (int ch = 0; ch < kChunks; ++ch) {
+                    const int c0 = c_begin + 16 * ch;
+                    if (c0 >= c_end) break;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        if (c0 + i >= t.n_rows) continue;
-                        __nv_bfloat16* o = out + (int64_t)(c0 + i) * p.ld_out;
-                        if constexpr (MODE == kGated) {
-                            o[0] = __float2bfloat16_rn(silu_mul(g[i], u[i]));
-                        } else {
-                            o[0] = __float2bfloat16_rn(g[i]);
-                            o[kBM] = __float2bfloat16_rn(u[i]);
-                        }
+                        if (c0 + i >= t.n_rows) break;
+                        uint16_t* o = out16 + (int64_t)(c0 + i) * p.ld_out;
+                        const int sh = 16 * (i & 1);
+                        o[0] = (uint16_t)(pk[ch][0][i >> 1] >> sh);
+                        if constexpr (kOut == 2) o[kBM] = (uint16_t)(pk[ch][1][i >> 1] >> sh);
                     }
-                } else {
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c0 + i < t.n_rows)
-                            out[(int64_t)(c0 + i) * p.ld_out] = __float2bfloat16_rn(g[i]);
                 }
+            } else {
+                for (int c0 = c_begin; c0 < c_end; c0 += 16) {
+                    float g[16];
+                    tmem_ld_16(tacc + c0, g);
+                    if constexpr (C::kNA == 2) {
+                        float u[16];
+                        tmem_ld_16(tacc + BN + c0, u);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            if (c0 + i >= t.n_rows) continue;
+                            __nv_bfloat16* o = out + (int64_t)(c0 + i) * p.ld_out;
+                            if constexpr (MODE == kGated) {
+                                o[0] = __float2bfloat16_rn(silu_mul(g[i], u[i]));
+                            } else {
+                                o[0] = __float2bfloat16_rn(g[i]);
+                                o[kBM] = __float2bfloat16_rn(u[i]);
+                            }
+                        }
+                    } else {
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < t.n_rows)
+                                out[(int64_t)(c0 + i) * p.ld_out] = __float2bfloat16_rn(g[i]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
             ++acc_use[acc];
             if (C::kAccBufs == 2) acc ^= 1;
         }

@@ -19,6 +19,13 @@ constexpr int kBoxN = 16;                      // token rows per TMA box
 constexpr uint32_t kABytes = kBM * kBK * 2;    // one weight tile, 16 KB
 constexpr uint32_t kSmemBudget = 200 * 1024;   // pipeline stages
 
+// K per pipeline stage of the bf16-operand kernel (kind::f16): 64 (128-byte
+// operand rows, 128-byte swizzle), or 32 (64-byte rows, 64-byte swizzle) for
+// e4m3 weights at 256-token tiles, where a 64-wide stage with its e4m3 staging
+// would leave room for two stages only.  The host encodes its tensor maps'
+// boxes with the same value.
+__host__ __device__ constexpr int stage_k(int bn, bool w8) { return (w8 && bn >= 256) ? 32 : kBK; }
+
 struct alignas(64) FfnArgs {
     CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}
     CUtensorMap act_map;       // activation rows {K, rows}, 16-row box
@@ -55,6 +62,13 @@ struct alignas(64) FfnArgs {
     uint32_t ready_epoch;
     int32_t slots_per_flag;
     uint64_t ready_timeout_ns;
+    // progress reports (NULL progress_word: none): when the d-th tile of this
+    // launch has its MMAs issued (d counted in *progress_tiles), the word is
+    // raised to progress_base + floor(d * progress_steps / tiles)
+    uint32_t* progress_word;
+    uint32_t* progress_tiles;
+    uint32_t progress_base;
+    int32_t progress_steps;
     // tile enumeration order: position i holds group order[i] (local experts
     // and the shared one first, then the remote experts in slot order, the
     // order in which a fetch fills them)
@@ -200,6 +214,31 @@ __device__ __forceinline__ bool gate_wait(const FfnArgs& p, int map, int slot, i
     asm volatile("fence.proxy.async.global;" ::: "memory");
     passed = f;
     return true;
+}
+
+// One more tile of this launch has its MMAs issued (called once per tile by
+// the MMA thread): count it, and when it completes a new step raise the
+// progress word to progress_base + step, a maximum in wrap-around order so
+// that a CTA that reports late never lowers it.
+__device__ __forceinline__ void report_progress(const FfnArgs& p, int total) {
+    if (!p.progress_word) return;
+    const uint64_t d = atomicAdd(p.progress_tiles, 1u) + 1ull;
+    const uint64_t steps = (uint64_t)p.progress_steps;
+    const uint32_t s = (uint32_t)(d * steps / (uint64_t)total);
+    if (s == (uint32_t)((d - 1) * steps / (uint64_t)total)) return;
+    const uint32_t v = p.progress_base + s;
+    uint32_t cur = *reinterpret_cast<volatile uint32_t*>(p.progress_word);
+    while ((int32_t)(v - cur) > 0) {
+        const uint32_t old = atomicCAS(p.progress_word, cur, v);
+        if (old == cur) break;
+        cur = old;
+    }
+}
+
+// Two fp32 values rounded to bf16 (round to nearest even), lo in bits 0-15.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&b);
 }
 
 // silu(g) * u = g / (1 + e^-g) * u with the fast exponential and division

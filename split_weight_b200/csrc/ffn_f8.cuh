@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(CfgF8<BN, MODE>::kThreads, 1)
                         phase ^= 1u;
                     }
                 }
+                if (ok) report_progress(p, total);
             }
         }
     } else {

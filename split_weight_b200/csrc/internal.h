@@ -53,6 +53,19 @@ moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t ra
                         const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                         CUtensorMapSwizzle swizzle);
 
+// Stream memory operations through the runtime's driver entry points
+// (cuStreamWriteValue32 / cuStreamWaitValue32; the 32-bit forms need no device
+// opt-in on CUDA 12).  The write lands once the stream's earlier work has
+// finished; the wait holds the stream until (int32_t)(*addr - value) >= 0.
+moe_status stream_write_u32(cudaStream_t s, uint32_t* addr, uint32_t value);
+moe_status stream_wait_geq_u32(cudaStream_t s, const uint32_t* addr, uint32_t value);
+
+// Progress value that releases chunk `chunk` of a paced fetch of n_chunks:
+// base for the first lead_chunks, the others spread evenly over the reports
+// base + 1 .. base + steps + 1 (moe_pace_threshold).
+uint32_t pace_threshold(int64_t chunk, int64_t n_chunks, int32_t lead_chunks, uint32_t base,
+                        int32_t steps);
+
 // Bits of the device error word.
 enum : int { kDevErrTimeout = 1, kDevErrIndex = 2 };
 

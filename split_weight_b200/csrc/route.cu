@@ -152,39 +152,33 @@ __global__ void __launch_bounds__(256) k_logits(const XT* __restrict__ x,
     }
 }
 
-// Large batches: a 64-token x 128-expert block tile, 4 x 8 (token, expert)
-// pairs per thread, 16 h per shared-memory stage with the next stage's
-// global loads held in registers while the current one is consumed.  The
-// arithmetic order is the same as k_logits: per 256-wide chunk a fused
-// multiply-add chain in ascending h, chunk sums added in ascending order.
+// Large batches: a 64-token x 128-expert block tile on 128 threads, 8 x 8
+// (token, expert) pairs per thread in packed fp32x2 fused multiply-adds
+// (four 16-byte shared loads feed 32 of them), 16 h per shared-memory stage
+// with the next stage's global loads held in registers while the current one
+// is consumed.  The arithmetic order is the same as k_logits: per 256-wide
+// chunk a fused multiply-add chain in ascending h, chunk sums added in
+// ascending order.
 constexpr int kBigT = 64, kBigE = 128, kBigK = 16;
 
 constexpr int kBigLd = kBigE + 4;  // row stride of the running sums in shared memory
 constexpr size_t kBigDynSmem = (size_t)kBigT * kBigLd * sizeof(float);
 
 template <typename XT>
-__global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
+__global__ void __launch_bounds__(128, 3) k_logits_big(const XT* __restrict__ x,
                                                        const float* __restrict__ wg, int T, int H,
                                                        int E, float* __restrict__ out) {
     __shared__ __align__(16) float xs[2][kBigK][kBigT + 4];  // [buffer][h][token]
     __shared__ __align__(16) float ws[2][kBigK][kBigE + 4];
-    extern __shared__ float ls[];  // [kBigT][kBigLd]: sum of the finished chunks, per pair
-    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    extern __shared__ float ls[];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;   // ty 0..7
     const int e0 = blockIdx.x * kBigE, t0 = blockIdx.y * kBigT;
-    // loader mapping: w  -> expert lt = tid / 2, h offset (tid % 2) * 8   (8 values)
-    //                 x  -> token  lt (threads with lt < 64 only)
-    // Two lanes share a row's 16 h.  Stored in step, their stage rows lh + i
-    // would sit 8 apart, and rows 8 apart hit the same banks at any 16-byte
-    // row stride.  The odd lane stores its values rotated by four: the pair
-    // writes rows i and 8 + (i + 4) % 8, 4 or 12 apart, which at a stride of
-    // 4 banks per row puts its 16 columns on the other 16 banks.
     const int lt = tid >> 1, lh = (tid & 1) * 8;
     const bool odd = tid & 1;
-    const bool xload = lt < kBigT;
-    const bool xin = xload && t0 + lt < T, win = e0 + lt < E;
+    const bool xin = t0 + lt < T, win = e0 + tid < E;
     const XT* xrow = x + (int64_t)(xin ? t0 + lt : 0) * H + lh;
-    const float* wrow = wg + (int64_t)(win ? e0 + lt : 0) * H + lh;
-    float rx[8], rw[8];
+    const float* wrow = wg + (int64_t)(win ? e0 + tid : 0) * H;
+    float rx[8], rw[16];
     auto load = [&](int h0) {
         if constexpr (sizeof(XT) == 2) {
             const uint4 u = xin ? *reinterpret_cast<const uint4*>(xrow + h0) : make_uint4(0, 0, 0, 0);
@@ -201,27 +195,31 @@ __global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
             rx[0] = a.x; rx[1] = a.y; rx[2] = a.z; rx[3] = a.w;
             rx[4] = b.x; rx[5] = b.y; rx[6] = b.z; rx[7] = b.w;
         }
-        const float4 a = win ? *reinterpret_cast<const float4*>(wrow + h0) : make_float4(0, 0, 0, 0);
-        const float4 b = win ? *reinterpret_cast<const float4*>(wrow + h0 + 4) : make_float4(0, 0, 0, 0);
-        rw[0] = a.x; rw[1] = a.y; rw[2] = a.z; rw[3] = a.w;
-        rw[4] = b.x; rw[5] = b.y; rw[6] = b.z; rw[7] = b.w;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 a = win ? *reinterpret_cast<const float4*>(wrow + h0 + 4 * q) : make_float4(0, 0, 0, 0);
+            rw[4 * q] = a.x; rw[4 * q + 1] = a.y; rw[4 * q + 2] = a.z; rw[4 * q + 3] = a.w;
+        }
     };
+    // x is staged transposed (h-major, rows of kBigT + 4 floats); the two
+    // lanes that load one token row write its column at h rows eight apart,
+    // which share a bank, so odd lanes store their eight rows rotated by four
+    // and a warp's stores hit 32 distinct banks
     auto store = [&](int buf) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int j = odd ? (i + 4) & 7 : i;
             const float vx = odd ? rx[(i + 4) & 7] : rx[i];
-            const float vw = odd ? rw[(i + 4) & 7] : rw[i];
-            if (xload) xs[buf][lh + j][lt] = vx;
-            ws[buf][lh + j][lt] = vw;
+            xs[buf][lh + j][lt] = vx;
         }
-    };
-    auto row_of = [&](int i) { return ty * 4 + i; };
-    auto col_of = [&](int j) { return j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4; };
-    // p[i][q] holds the chain sums of columns col_of(2q), col_of(2q + 1)
-    uint64_t p[4][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 16; ++i) ws[buf][i][tid] = rw[i];
+    };
+    auto row_of = [&](int i) { return i < 4 ? ty * 4 + i : 32 + ty * 4 + i - 4; };
+    auto col_of = [&](int j) { return j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4; };
+    uint64_t p[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int q = 0; q < 4; ++q) p[i][q] = 0;
     const int nk = H / kBigK;
@@ -234,23 +232,24 @@ __global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
 #pragma unroll
         for (int kk = 0; kk < kBigK; ++kk) {
             const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][kk][32 + ty * 4]);
             const float4 b0 = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * 4]);
             const float4 b1 = *reinterpret_cast<const float4*>(&ws[buf][kk][64 + tx * 4]);
-            const float a[4] = {a0.x, a0.y, a0.z, a0.w};
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const uint64_t b[4] = {pack2(b0.x, b0.y), pack2(b0.z, b0.w), pack2(b1.x, b1.y),
                                    pack2(b1.z, b1.w)};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 8; ++i) {
                 const uint64_t ai = pack2(a[i], a[i]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) fma2(p[i][q], ai, b[q]);
             }
         }
         const int h_next = (kt + 1) * kBigK;
-        if (h_next % kChunk == 0 || h_next >= H) {  // a 256-wide chunk ends here
+        if (h_next % kChunk == 0 || h_next >= H) {
             const bool first = (h_next - 1) / kChunk == 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float2 v = unpack2(p[i][q]);
@@ -265,7 +264,7 @@ __global__ void __launch_bounds__(256, 2) k_logits_big(const XT* __restrict__ x,
         __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
         const int t = t0 + row_of(i);
         if (t >= T) continue;
 #pragma unroll
@@ -527,7 +526,7 @@ void launch_logits(const moe_route_cfg* c, const RoutePlan& p, const XT* x, cons
         dim3 g((c->E + kBigE - 1) / kBigE, (c->T + kBigT - 1) / kBigT);
         cudaFuncSetAttribute(k_logits_big<XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kBigDynSmem);
-        k_logits_big<XT><<<g, 256, kBigDynSmem, s>>>(x, wg, c->T, c->H, c->E, out);
+        k_logits_big<XT><<<g, 128, kBigDynSmem, s>>>(x, wg, c->T, c->H, c->E, out);
     } else if (p.tm == 2) {
         k_logits<XT, 2, 2><<<grid, 256, 0, s>>>(x, wg, c->T, c->H, c->E, p.nsplit > 1, out);
     } else {

@@ -142,6 +142,19 @@ class ReadyGate:
                                 self.slots_per_flag, self.flags.numel(), self.timeout_ns)
 
 
+@dataclass
+class Progress:
+    """Progress reports of a grouped-GEMM call (moe_progress): words[0] is
+    the progress word, words[1:3] the call's tile counters."""
+    words: torch.Tensor          # int32 [3] on the device (read as uint32)
+    base: int
+    steps: int
+
+    def c_struct(self) -> L.moe_progress:
+        w = self.words.data_ptr()
+        return L.moe_progress(w, w + 4, self.base & 0xFFFFFFFF, self.steps)
+
+
 class MoELayer:
     """One MoE layer with preallocated device buffers.
 
@@ -204,13 +217,25 @@ class MoELayer:
                               self.perm_ws.data_ptr(), self.perm_ws.numel(), stream))
 
     def grouped_ffn(self, stream: int, remote: torch.Tensor | None = None,
-                    gate: "ReadyGate | None" = None, x: torch.Tensor | None = None) -> None:
+                    gate: "ReadyGate | None" = None, x: torch.Tensor | None = None,
+                    progress: Progress | None = None) -> None:
         """The grouped GEMMs; with a gate, remote experts are read only once
         their chunk of a fetch still in flight has landed.  x: the layer
-        input, needed when the token rows are gathered from it."""
+        input, needed when the token rows are gathered from it.  progress:
+        reports that pace a fetch (moe_grouped_ffn_paced)."""
         tbl = self.weights.table(remote)
         g = gate.c_struct() if gate is not None else None
         gp = ctypes.byref(g) if g is not None else None
+        if progress is not None:
+            pr = progress.c_struct()
+            xp = x.data_ptr() if self.gather else None
+            ps = self.perm_src.data_ptr() if self.gather else None
+            L.check(L.moe_grouped_ffn_paced(ctypes.byref(self._desc), ctypes.byref(tbl), gp,
+                                            ctypes.byref(pr), _ptr(self.x_perm), _ptr(self.x_scales),
+                                            xp, ps, self.offsets.data_ptr(), self.h.data_ptr(),
+                                            self.y_perm.data_ptr(), self.ffn_ws.data_ptr(),
+                                            self.ffn_ws.numel(), stream))
+            return
         if self.gather:
             assert x is not None, "the gathered grouped GEMM reads the layer input x"
             L.check(L.moe_grouped_ffn_x(ctypes.byref(self._desc), ctypes.byref(tbl), gp,
@@ -271,12 +296,22 @@ class PrefetchPipeline:
     window_block(l, x, stream), if given, is enqueued before layer l's MoE
     block: compute that the fetch also hides behind (the explainer's
     attention block between two MoE blocks).
+
+    With pace_steps > 0 (and gate_slots > 0) the fetch is paced by compute:
+    execution g enqueues the fetch of execution g + 1 just before its own
+    grouped GEMM call, which reports its progress in pace_steps steps
+    (moe_grouped_ffn_paced, base g' (pace_steps + 1) for the g'-th paced
+    execution); the first pace_lead chunks go at once, the others wait on
+    the copy stream for an even share of those reports
+    (moe_prefetch_layer_paced).  The copy then runs spread over the grouped
+    GEMMs instead of as one burst beside them, and a fetch never waits on a
+    call that is not enqueued yet.
     """
 
     def __init__(self, layers: list[MoELayer], peer_stores: list[torch.Tensor],
                  remote_bytes: int, device: torch.device | str = "cuda", chunk_bytes: int = 0,
                  split: bool = True, gate_slots: int = 0, window_block=None,
-                 gate_timeout_ns: int = 0):
+                 gate_timeout_ns: int = 0, pace_steps: int = 0, pace_lead: int = 0):
         self.layers, self.peer_stores = layers, peer_stores
         self.remote_bytes, self.chunk_bytes = remote_bytes, chunk_bytes
         self.split, self.pending = split, None
@@ -292,14 +327,23 @@ class PrefetchPipeline:
         self.g = 0
         self.stride = layers[0].weights.stride
         self.flags = None
-        self.configure(gate_slots=gate_slots)
+        self.pace_steps, self.pace_lead, self.g_pace0 = 0, 0, 0
+        self.progress_words = torch.zeros(3, dtype=torch.int32, device=dev)
+        self.configure(gate_slots=gate_slots, pace_steps=pace_steps, pace_lead=pace_lead)
 
     def configure(self, split: bool | None = None, gate_slots: int | None = None,
-                  window_block=False) -> None:
+                  window_block=False, pace_steps: int | None = None,
+                  pace_lead: int | None = None) -> None:
         """Switches the schedule between runs (after a synchronisation: no
         fetch may be in flight).  window_block=False leaves it as it is."""
         if split is not None:
             self.split = split
+        if pace_lead is not None:
+            self.pace_lead = pace_lead
+        if pace_steps is not None:
+            self.pace_steps = pace_steps
+            self.g_pace0 = self.g
+            self.progress_words.zero_()   # the base of execution g_pace0
         if window_block is not False:
             self.window_block = window_block
         if gate_slots is not None:
@@ -312,15 +356,32 @@ class PrefetchPipeline:
                 # flags only grow: fresh zeros are below every epoch still to come
                 self.flags = [torch.zeros(self.n_flags, dtype=torch.int32, device=dev)
                               for _ in range(2)]
+        if self.pace_steps > 0:
+            assert self.gate_slots > 0 and self.pace_steps >= 2, \
+                "a paced fetch needs readiness flags and at least 2 steps"
         self.pending = None
 
+    def progress(self, execution: int) -> Progress:
+        """The progress reports of a paced execution's grouped GEMM call."""
+        return Progress(self.progress_words, (execution - self.g_pace0) * (self.pace_steps + 1),
+                        self.pace_steps)
+
     # -- copies -------------------------------------------------------------
-    def _copy(self, layer: int, buf: int, lo: int, hi: int, wait_free, ready, epoch: int) -> None:
+    def _copy(self, layer: int, buf: int, lo: int, hi: int, wait_free, ready, epoch: int,
+              pace: Progress | None = None) -> None:
         src = self.peer_stores[layer].data_ptr() + lo
         dst = self.bufs[buf].data_ptr() + lo
         wf = wait_free.cuda_event if wait_free is not None else None
         rd = ready.cuda_event if ready is not None else None
-        if self.gate_slots > 0:
+        if pace is not None:
+            chunk = self.gate_slots * self.stride
+            pr = pace.c_struct()
+            L.check(L.moe_prefetch_layer_paced(src, dst, hi - lo, chunk,
+                                               self.copy_stream.cuda_stream, wf,
+                                               self.flags[buf].data_ptr() + 4 * (lo // chunk),
+                                               epoch & 0xFFFFFFFF, ctypes.byref(pr),
+                                               self.pace_lead, rd))
+        elif self.gate_slots > 0:
             chunk = self.gate_slots * self.stride
             assert lo % chunk == 0
             L.check(L.moe_prefetch_layer_flagged(src, dst, hi - lo, chunk,
@@ -354,10 +415,11 @@ class PrefetchPipeline:
         self._copy(layer, buf, lo, hi, wait_free, self.ready[buf] if half == 1 else None, ex + 1)
 
     def prime(self) -> None:
-        """Enqueues the fetches of the next two executions (before a run)."""
+        """Enqueues the fetches of the next two executions (before a run);
+        paced, of the next one (each execution enqueues its successor's)."""
         n = len(self.layers)
         self.pending = None
-        for i in range(2):
+        for i in range(1 if self.pace_steps > 0 else 2):
             self.prefetch((self.g + i) % n, (self.g + i) % 2, None, self.g + i)
 
     # -- compute ------------------------------------------------------------
@@ -376,12 +438,21 @@ class PrefetchPipeline:
             gate = ReadyGate(self.flags[b], g + 1, self.gate_slots, self.gate_timeout_ns)
         elif prefetch:
             stream.wait_event(self.ready[b])
+        progress = None
+        if prefetch and self.pace_steps > 0:
+            progress = self.progress(g)
+            if l + 1 < n or wrap:   # execution g + 1's fetch, paced by this call
+                nb = (g + 1) % 2
+                self._copy((l + 1) % n, nb, 0, self.remote_bytes, self.free[nb], self.ready[nb],
+                           g + 2, pace=progress)
         if ffn_events is not None:
             ffn_events[0].record(stream)
-        layer.grouped_ffn(h, self.bufs[b], gate, x=x)
+        layer.grouped_ffn(h, self.bufs[b], gate, x=x, progress=progress)
         if ffn_events is not None:
             ffn_events[1].record(stream)
-        if prefetch and self.split:
+        if progress is not None:
+            self.free[b].record(stream)
+        elif prefetch and self.split:
             self.free[b].record(stream)
             if self.pending is not None:  # second half of execution g + 1's fetch
                 self.fetch_half(*self.pending, 1, self.free[b], g + 1)

@@ -65,10 +65,18 @@ class FakeLayer:
     def permute(self, x, h):
         pass
 
-    def grouped_ffn(self, h, remote, gate=None, x=None):
+    def grouped_ffn(self, h, remote, gate=None, x=None, progress=None):
         if gate is not None:   # the gated kernel reads each chunk once its flag reached the epoch
             Log.ops.append(("gate", "compute", gate.flags.owner, gate.epoch))
+        if progress is not None:
+            # reports while the GEMMs still read their buffer: logged before the
+            # read, so a paced chunk released by them that touched this buffer
+            # would show in the snapshot
+            for st in range(1, progress.steps + 1):
+                Log.ops.append(("progress", "compute", progress.base + st))
         Log.ops.append(("ffn", "compute", self.idx, remote.owner))
+        if progress is not None:   # the call's final write
+            Log.ops.append(("progress", "compute", progress.base + progress.steps + 1))
 
     def combine(self, h):
         pass
@@ -101,6 +109,29 @@ def fake_prefetch_flagged(src, dst, nbytes, chunk, stream, wait, flags, epoch, r
     return L.MOE_OK
 
 
+def fake_prefetch_paced(src, dst, nbytes, chunk, stream, wait, flags, epoch, pace, lead, ready):
+    if wait is not None:
+        ev = FakeEvent.by_id[wait]
+        Log.ops.append(("wait", "copy", ev, ev.version))
+    assert src[1] == dst[1] and src[1] % chunk == 0
+    first = src[1] // chunk
+    assert flags[1] == 4 * first
+    n = -(-nbytes // chunk)
+    for i, lo in enumerate(range(src[1], src[1] + nbytes, chunk)):
+        hi = min(lo + chunk, src[1] + nbytes)
+        Log.ops.append(("pwait", "copy", L.moe_pace_threshold(i, n, lead, pace.base, pace.steps)))
+        Log.ops.append(("copy", "copy", src[0], dst[0], lo, hi))
+        Log.ops.append(("flag", "copy", flags[0], first + i, epoch))
+    if ready is not None:
+        FakeEvent.by_id[ready].record(FakeStream(name="copy"))
+    return L.MOE_OK
+
+
+class FakeProgress:
+    def __init__(self, word, tiles, base, steps):
+        self.word, self.tiles, self.base, self.steps = word, tiles, base, steps
+
+
 class FlagBuffer(Buffer):
     def __init__(self, owner, n):
         super().__init__(owner)
@@ -116,7 +147,7 @@ def replay(ops, nbytes, n_flags=0):
     done = {}  # event id -> highest executed record version
     queues = {s: [o for o in ops if o[1] == s] for s in ("compute", "copy")}
     pos = {s: 0 for s in queues}
-    buffers, seen, moved, flags = {}, [], True, {}
+    buffers, seen, moved, flags, word = {}, [], True, {}, 0
     while moved:
         moved = False
         for s, q in queues.items():
@@ -126,6 +157,11 @@ def replay(ops, nbytes, n_flags=0):
                     break
                 if op[0] == "gate" and any(flags.get((op[2], c), 0) < op[3] for c in range(n_flags)):
                     break
+                if op[0] == "pwait" and ((word - op[2]) & 0xFFFFFFFF) >= 1 << 31:
+                    break   # (int32_t)(word - threshold) < 0
+                if op[0] == "progress":
+                    if ((op[2] - word) & 0xFFFFFFFF) < 1 << 31:
+                        word = op[2]
                 if op[0] == "flag":
                     flags[(op[2], op[3])] = op[4]
                 if op[0] == "record":
@@ -142,19 +178,31 @@ def replay(ops, nbytes, n_flags=0):
     return seen
 
 
+@pytest.mark.parametrize("pace", [(0, 0), (3, 0), (3, 1), (2, 5)],
+                         ids=["unpaced", "paced", "paced_lead1", "paced_all_lead"])
 @pytest.mark.parametrize("gate_slots", [0, 2], ids=["events", "flags"])
 @pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
 @pytest.mark.parametrize("n_layers", [1, 2, 3, 4])
-def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_layers, gate_slots):
+def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_layers, gate_slots,
+                                                         pace):
     """Event-gated schedule: the compute stream waits for ready.  Flag-gated
     schedule: the grouped GEMM of execution g waits on the device for every
     chunk flag of its buffer to reach g + 1; each flag must be written only
     after its chunk holds the right layer, and never for a later fetch before
-    the grouped GEMM that needs the earlier one has run."""
+    the grouped GEMM that needs the earlier one has run.  Paced schedule
+    (flags, pace_steps > 0): each chunk of execution g + 1's fetch also
+    waits on the copy stream for execution g's progress reports; no wait
+    may be left without the call that satisfies it."""
+    pace_steps, pace_lead = pace
+    if pace_steps and not gate_slots:
+        pytest.skip("a paced fetch needs readiness flags")
     monkeypatch.setattr(torch.cuda, "Stream", FakeStream)
     monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
     monkeypatch.setattr(L, "moe_prefetch_layer", fake_prefetch)
     monkeypatch.setattr(L, "moe_prefetch_layer_flagged", fake_prefetch_flagged)
+    monkeypatch.setattr(L, "moe_prefetch_layer_paced", fake_prefetch_paced)
+    monkeypatch.setattr(L, "moe_progress", FakeProgress)
+    monkeypatch.setattr(layer_mod.ctypes, "byref", lambda o: o)
     monkeypatch.setattr(L, "check", lambda status: None)
     Log.ops = []
     # events: an odd size (the halves split at a 256-byte boundary); flags:
@@ -180,6 +228,8 @@ def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_l
     for ev in pipe.ready + pipe.free:
         ev.record(pipe.copy_stream)
     pipe.g = 0
+    pipe.pace_steps, pipe.pace_lead, pipe.g_pace0 = pace_steps, pace_lead, 0
+    pipe.progress_words = Buffer(("progress", 0))
 
     compute = FakeStream(name="compute")
     pipe.prime()
