@@ -459,16 +459,18 @@ MOE_API moe_status moe_prefetch_layer_flagged(const void *src, void *dst, size_t
                                       cudaEvent_t ready_out);
 
 /* moe_prefetch_layer_flagged paced by a grouped-GEMM call's progress (see
- * moe_progress): before chunk c of n the copy stream waits until
+ * moe_progress): before chunk c of n a one-thread kernel on the copy stream
+ * waits until
  *   (int32_t)(*pace->word - moe_pace_threshold(c, n, lead_chunks, pace->base,
  *                                              pace->steps)) >= 0
- * (cuStreamWaitValue32, no SM involved).  The first lead_chunks chunks go at
- * once; the others are spread evenly over the call's reports, the last one
- * released by report base + steps.  The pacing call must be enqueued on its
- * stream (or already have run) when the copy stream gets there, or the copy
- * stream waits for it: issue the fetch and the call together.  Only the
- * word is read (pace->tiles unused).  MOE_ERR_UNSUPPORTED if the driver
- * lacks cuStreamWaitValue32 or cuStreamWriteValue32. */
+ * or 200 ms have passed, whichever comes first (a wait that runs out lets
+ * the chunk go: pacing spreads the copy, the flags order it).  The first
+ * lead_chunks chunks go at once; the others are spread evenly over the
+ * call's reports, the last one released by report base + steps.  Enqueue
+ * the pacing call BEFORE this fetch: streams may share a hardware queue, and
+ * a wait queued ahead of its call would then hold the call back until it
+ * runs out.  Only the word is read (pace->tiles unused).
+ * MOE_ERR_UNSUPPORTED if the driver lacks cuStreamWriteValue32. */
 MOE_API moe_status moe_prefetch_layer_paced(const void *src, void *dst, size_t bytes,
                                     size_t chunk_bytes, cudaStream_t copy_stream,
                                     cudaEvent_t wait_free, uint32_t *flags, uint32_t epoch,

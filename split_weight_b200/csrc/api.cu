@@ -6,6 +6,7 @@
 #include <mutex>
 #include <thread>
 
+#include "device.cuh"
 #include "internal.h"
 
 namespace swb {
@@ -113,7 +114,7 @@ moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t ra
 
 using StreamValue32Fn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
 namespace {
-StreamValue32Fn g_write32 = nullptr, g_wait32 = nullptr;
+StreamValue32Fn g_write32 = nullptr;
 
 moe_status stream_value_fn(const char* name, StreamValue32Fn* cache, StreamValue32Fn* out) {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -143,22 +144,31 @@ moe_status stream_write_u32(cudaStream_t s, uint32_t* addr, uint32_t value) {
     return MOE_OK;
 }
 
-moe_status stream_wait_geq_u32(cudaStream_t s, const uint32_t* addr, uint32_t value) {
-    StreamValue32Fn fn = nullptr;
-    moe_status st = stream_value_fn("cuStreamWaitValue32", &g_wait32, &fn);
-    if (st != MOE_OK) return st;
-    if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "cuStreamWaitValue32: injected failure");
-    const CUresult r = fn(reinterpret_cast<CUstream>(s), reinterpret_cast<CUdeviceptr>(addr), value,
-                          CU_STREAM_WAIT_VALUE_GEQ);
-    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuStreamWaitValue32 failed (CUresult %d)", (int)r);
-    return MOE_OK;
-}
 
 uint32_t pace_threshold(int64_t chunk, int64_t n_chunks, int32_t lead_chunks, uint32_t base,
                         int32_t steps) {
     if (chunk < lead_chunks) return base;
     const int64_t paced = n_chunks - lead_chunks, j = chunk - lead_chunks;
     return base + (uint32_t)(((j + 1) * ((int64_t)steps + 1)) / (paced + 1));
+}
+
+// A paced chunk's wait, one thread on the copy stream: polls the progress
+// word (acquire loads at GPU scope) until it reaches the threshold, or gives
+// up after kPaceWaitNs and lets the chunk go (pacing only spreads the copy;
+// the readiness flags, not this wait, order it before its readers).  A
+// bounded kernel rather than a stream memory wait, so that no ordering of
+// streams on the hardware queues can turn it into a wait without end.
+constexpr uint64_t kPaceWaitNs = 200000000ull;   // 200 ms
+
+__global__ void k_pace_wait(const uint32_t* word, uint32_t threshold, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(word) : "memory");
+        if ((int32_t)(v - threshold) >= 0) return;
+        if (globaltimer_ns() - t0 > limit_ns) return;
+        __nanosleep(2000);
+    }
 }
 
 // The chunked copy of moe_prefetch_layer_flagged / _paced: per chunk an
@@ -172,10 +182,14 @@ moe_status flagged_copy(const void* src, void* dst, size_t bytes, size_t chunk_b
     int64_t c = 0;
     for (size_t off = 0; off < bytes; off += chunk_bytes, ++c) {
         moe_status st;
-        if (pace && (st = stream_wait_geq_u32(copy_stream, pace->word,
-                                              pace_threshold(c, n, lead_chunks, pace->base,
-                                                             pace->steps))) != MOE_OK)
-            return st;
+        if (pace) {
+            const uint32_t thr = pace_threshold(c, n, lead_chunks, pace->base, pace->steps);
+            if (thr != pace->base) {   // the lead chunks go at once
+                if (cuda_injected_failure()) return fail(MOE_ERR_CUDA, "k_pace_wait: injected failure");
+                k_pace_wait<<<1, 1, 0, copy_stream>>>(pace->word, thr, kPaceWaitNs);
+                SWB_LAUNCHED("k_pace_wait");
+            }
+        }
         const size_t len = bytes - off < chunk_bytes ? bytes - off : chunk_bytes;
         SWB_CUDA(cudaMemcpyAsync(static_cast<char*>(dst) + off,
                                  static_cast<const char*>(src) + off, len,

@@ -53,12 +53,10 @@ moe_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t ra
                         const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                         CUtensorMapSwizzle swizzle);
 
-// Stream memory operations through the runtime's driver entry points
-// (cuStreamWriteValue32 / cuStreamWaitValue32; the 32-bit forms need no device
-// opt-in on CUDA 12).  The write lands once the stream's earlier work has
-// finished; the wait holds the stream until (int32_t)(*addr - value) >= 0.
+// cuStreamWriteValue32 through the runtime's driver entry point (the 32-bit
+// stream memory operations need no device opt-in on CUDA 12): the write lands
+// once the stream's earlier work has finished.
 moe_status stream_write_u32(cudaStream_t s, uint32_t* addr, uint32_t value);
-moe_status stream_wait_geq_u32(cudaStream_t s, const uint32_t* addr, uint32_t value);
 
 // Progress value that releases chunk `chunk` of a paced fetch of n_chunks:
 // base for the first lead_chunks, the others spread evenly over the reports

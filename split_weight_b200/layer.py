@@ -298,14 +298,13 @@ class PrefetchPipeline:
     attention block between two MoE blocks).
 
     With pace_steps > 0 (and gate_slots > 0) the fetch is paced by compute:
-    execution g enqueues the fetch of execution g + 1 just before its own
-    grouped GEMM call, which reports its progress in pace_steps steps
-    (moe_grouped_ffn_paced, base g' (pace_steps + 1) for the g'-th paced
-    execution); the first pace_lead chunks go at once, the others wait on
-    the copy stream for an even share of those reports
-    (moe_prefetch_layer_paced).  The copy then runs spread over the grouped
-    GEMMs instead of as one burst beside them, and a fetch never waits on a
-    call that is not enqueued yet.
+    right after enqueuing its grouped GEMM call, which reports its progress
+    in pace_steps steps (moe_grouped_ffn_paced, base g' (pace_steps + 1) for
+    the g'-th paced execution), execution g enqueues the fetch of execution
+    g + 1; its first pace_lead chunks go at once, the others wait on the copy
+    stream for an even share of those reports (moe_prefetch_layer_paced).
+    The copy then runs spread over the grouped GEMMs instead of as one burst
+    beside them, and never waits for work enqueued after it.
     """
 
     def __init__(self, layers: list[MoELayer], peer_stores: list[torch.Tensor],
@@ -316,7 +315,7 @@ class PrefetchPipeline:
         self.remote_bytes, self.chunk_bytes = remote_bytes, chunk_bytes
         self.split, self.pending = split, None
         self.gate_slots, self.window_block, self.gate_timeout_ns = gate_slots, window_block, gate_timeout_ns
-        dev = torch.device(device)
+        dev = self.device = torch.device(device)
         self.bufs = [torch.empty(max(remote_bytes, 1), dtype=torch.uint8, device=dev)
                      for _ in range(2)]
         self.copy_stream = torch.cuda.Stream(device=dev)
@@ -416,8 +415,12 @@ class PrefetchPipeline:
 
     def prime(self) -> None:
         """Enqueues the fetches of the next two executions (before a run);
-        paced, of the next one (each execution enqueues its successor's)."""
+        paced, of the next one (each execution enqueues its successor's).
+        The copy stream first waits for the current stream: the flags and
+        progress words that configure() zero-filled there, and the peer
+        stores, must be in place before a fetch writes or reads them."""
         n = len(self.layers)
+        self.copy_stream.wait_stream(torch.cuda.current_stream(self.device))
         self.pending = None
         for i in range(1 if self.pace_steps > 0 else 2):
             self.prefetch((self.g + i) % n, (self.g + i) % 2, None, self.g + i)
@@ -438,13 +441,7 @@ class PrefetchPipeline:
             gate = ReadyGate(self.flags[b], g + 1, self.gate_slots, self.gate_timeout_ns)
         elif prefetch:
             stream.wait_event(self.ready[b])
-        progress = None
-        if prefetch and self.pace_steps > 0:
-            progress = self.progress(g)
-            if l + 1 < n or wrap:   # execution g + 1's fetch, paced by this call
-                nb = (g + 1) % 2
-                self._copy((l + 1) % n, nb, 0, self.remote_bytes, self.free[nb], self.ready[nb],
-                           g + 2, pace=progress)
+        progress = self.progress(g) if prefetch and self.pace_steps > 0 else None
         if ffn_events is not None:
             ffn_events[0].record(stream)
         layer.grouped_ffn(h, self.bufs[b], gate, x=x, progress=progress)
@@ -452,6 +449,13 @@ class PrefetchPipeline:
             ffn_events[1].record(stream)
         if progress is not None:
             self.free[b].record(stream)
+            # execution g + 1's fetch, paced by the call just enqueued: the
+            # call goes first, so that the copy stream never waits for work
+            # queued behind it (streams may share a hardware queue)
+            if l + 1 < n or wrap:
+                nb = (g + 1) % 2
+                self._copy((l + 1) % n, nb, 0, self.remote_bytes, self.free[nb], self.ready[nb],
+                           g + 2, pace=progress)
         elif prefetch and self.split:
             self.free[b].record(stream)
             if self.pending is not None:  # second half of execution g + 1's fetch

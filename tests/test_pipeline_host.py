@@ -39,6 +39,9 @@ class FakeStream:
     def wait_event(self, ev):
         Log.ops.append(("wait", self.name, ev, ev.version))
 
+    def wait_stream(self, other):   # ordering against the caller's earlier work
+        pass
+
 
 class Ptr(tuple):
     """A device pointer stand-in: (owner, byte offset)."""
@@ -141,11 +144,16 @@ class FlagBuffer(Buffer):
         return self.n
 
 
-def replay(ops, nbytes, n_flags=0):
+def replay(ops, nbytes, n_flags=0, shared=False):
     """Runs both streams in order, honouring waits; returns (layer, buffer
-    contents) for every grouped GEMM in execution order."""
+    contents) for every grouped GEMM in execution order.  shared=True runs
+    both streams' work as one hardware queue in host order (streams that
+    share a queue): a wait then blocks everything enqueued after it."""
     done = {}  # event id -> highest executed record version
-    queues = {s: [o for o in ops if o[1] == s] for s in ("compute", "copy")}
+    if shared:
+        queues = {"all": list(ops)}
+    else:
+        queues = {s: [o for o in ops if o[1] == s] for s in ("compute", "copy")}
     pos = {s: 0 for s in queues}
     buffers, seen, moved, flags, word = {}, [], True, {}, 0
     while moved:
@@ -191,8 +199,9 @@ def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_l
     after its chunk holds the right layer, and never for a later fetch before
     the grouped GEMM that needs the earlier one has run.  Paced schedule
     (flags, pace_steps > 0): each chunk of execution g + 1's fetch also
-    waits on the copy stream for execution g's progress reports; no wait
-    may be left without the call that satisfies it."""
+    waits on the copy stream for execution g's progress reports.  Every
+    schedule must also complete when both streams share one hardware queue,
+    i.e. no wait is enqueued ahead of the work that satisfies it."""
     pace_steps, pace_lead = pace
     if pace_steps and not gate_slots:
         pytest.skip("a paced fetch needs readiness flags")
@@ -230,19 +239,22 @@ def test_every_grouped_gemm_reads_its_own_complete_fetch(monkeypatch, split, n_l
     pipe.g = 0
     pipe.pace_steps, pipe.pace_lead, pipe.g_pace0 = pace_steps, pace_lead, 0
     pipe.progress_words = Buffer(("progress", 0))
+    pipe.device = None
 
     compute = FakeStream(name="compute")
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: compute)
     pipe.prime()
     n_exec = 3 * n_layers + 1
     for i in range(n_exec):
         pipe.run_layer(i % n_layers, None, compute, prefetch=True, wrap=True)
 
-    seen = replay(Log.ops, nbytes, n_flags)
-    assert len(seen) == n_exec
-    for i, (lidx, content) in enumerate(seen):
-        assert lidx == i % n_layers
-        assert all(c == ("store", lidx) for c in content), (
-            f"execution {i} (layer {lidx}) read {sorted(set(map(str, content)))}")
+    for shared in (False, True):   # independent queues, then one shared queue
+        seen = replay(Log.ops, nbytes, n_flags, shared)
+        assert len(seen) == n_exec
+        for i, (lidx, content) in enumerate(seen):
+            assert lidx == i % n_layers
+            assert all(c == ("store", lidx) for c in content), (
+                f"execution {i} (layer {lidx}) read {sorted(set(map(str, content)))}")
 
 
 def test_split_halves_cover_the_buffer_once(monkeypatch):
