@@ -427,6 +427,9 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
       flags_paced     flags, the fetch of the next execution issued before
                       each grouped GEMM call and paced by its progress
                       reports (24 steps, 2 chunks ahead)
+      selective       per-slot flags; only the remote slots predicted by a
+                      look-ahead routing (the next layer's router on this
+                      layer's input), then the ones it missed
       window_*        the same schedules with a dense compute block
                       (R1 attention FLOPs) before every MoE block, the
                       explainer's two-block window; its no-copy baseline runs
@@ -435,15 +438,17 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
     import torch
     from split_weight_b200 import DenseBlock
     from split_weight_b200 import _lib as L
-    saved = (pipe.split, pipe.gate_slots, pipe.window_block, pipe.pace_steps, pipe.pace_lead)
+    saved = (pipe.split, pipe.gate_slots, pipe.window_block, pipe.pace_steps, pipe.pace_lead,
+             pipe.select)
     steps = max(3, args.workload_steps)
 
-    def run(split, gate_slots, window, pace_steps=0, pace_lead=2):
+    def run(split, gate_slots, window, pace_steps=0, pace_lead=2, select=False):
         """One schedule; a kernel wait that ran out (or another device
         check) is reported in its entry, not raised."""
         torch.cuda.synchronize()
         pipe.configure(split=split, gate_slots=gate_slots, window_block=window,
-                       pace_steps=pace_steps, pace_lead=pace_lead)
+                       pace_steps=pace_steps, pace_lead=pace_lead, select=select)
+        pipe.select_stats = []
         pipe.prime()
         for _ in range(2):
             step()
@@ -460,15 +465,30 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
         st = L.moe_check_device()
         if st != L.MOE_OK:
             return {"error": f"{L.status_string(st)}: {L.moe_last_error()}"}
+        stats = list(pipe.select_stats)
         out = prefetch_overlap(cfg, pipe, step, stream, e0.elapsed_time(e1) / steps, steps)
         out.pop("_ffn_ms_no_copy", None)
+        if select and stats:   # remote slots fetched per execution, after the first pass
+            later = stats[cfg.layers:] or stats
+            n_slots = pipe.remote_bytes // pipe.stride
+            out["selective"] = {
+                "remote_slots": n_slots,
+                "touched_per_layer": round(float(np.mean([x["touched"] for x in later])), 2),
+                "predicted_per_layer": round(float(np.mean([x.get("predicted_next", 0)
+                                                            for x in later])), 2),
+                "missed_per_layer": round(float(np.mean([x["missed"] for x in later])), 2),
+            }
+            f = out["selective"]
+            f["fetched_fraction"] = round((f["predicted_per_layer"] + f["missed_per_layer"])
+                                          / n_slots, 4)
         st = L.moe_check_device()
         if st != L.MOE_OK:
             out["error"] = f"{L.status_string(st)} in the no-copy or copy-alone runs"
         return out
 
     out = {"events_halves": run(True, 0, None), "flags_whole": run(False, 8, None),
-           "flags_halves": run(True, 8, None), "flags_paced": run(False, 8, None, 24, 2)}
+           "flags_halves": run(True, 8, None), "flags_paced": run(False, 8, None, 24, 2),
+           "selective": run(False, 1, None, select=True)}
     if args.window_inter > 0:
         block = DenseBlock(cfg.T, cfg.H, args.window_inter, dev)
         out["window_block"] = {"inter": args.window_inter,
@@ -479,7 +499,7 @@ def prefetch_schedules(cfg, pipe, step, stream, args, dev):
         del block
     torch.cuda.synchronize()
     pipe.configure(split=saved[0], gate_slots=saved[1], window_block=saved[2],
-                   pace_steps=saved[3], pace_lead=saved[4])
+                   pace_steps=saved[3], pace_lead=saved[4], select=saved[5])
     pipe.prime()
     torch.cuda.synchronize()
     return out

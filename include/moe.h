@@ -485,6 +485,33 @@ MOE_API moe_status moe_prefetch_layer_paced(const void *src, void *dst, size_t b
 MOE_API uint32_t moe_pace_threshold(int64_t chunk, int64_t n_chunks, int32_t lead_chunks,
                                     uint32_t base, int32_t steps);
 
+/* Selective prefetch (the predicted-routing prefetch of the offloading
+ * diagram on the pages; this library's reading: fetch only the remote experts
+ * a layer is predicted to touch, then the ones the prediction missed).
+ * Copies slots[0 .. n) of a remote pool image of pool_slots slots, slot s
+ * being the slot_bytes at offset s * slot_bytes of src and of dst (both
+ * pool_slots * slot_bytes long, not overlapping); a run of consecutive
+ * indices is one cudaMemcpyAsync, after which the copy stream writes
+ * flags[s] = epoch for each slot s of the run (per-slot readiness: a
+ * moe_ready_gate with slots_per_flag = 1, n_flags = pool_slots).
+ * slots: host array, values in [0, pool_slots) (else MOE_ERR_INVALID_ARG
+ * before anything is enqueued); flags: device, pool_slots words, 4-byte
+ * aligned.  wait_free / ready_out as for moe_prefetch_layer.  n = 0 copies
+ * nothing. */
+MOE_API moe_status moe_prefetch_slots(const void *src, void *dst, size_t slot_bytes,
+                              int32_t pool_slots, const int32_t *slots, int32_t n,
+                              cudaStream_t copy_stream, cudaEvent_t wait_free, uint32_t *flags,
+                              uint32_t epoch, cudaEvent_t ready_out);
+
+/* The experts a routing selects: touched[e] = 1 if some entry of topk_idx
+ * [A] equals e, else 0 (touched: device, E bytes, zeroed by the call on
+ * `stream`).  Entries outside [0, E) are reported through the device error
+ * word (MOE_ERR_DEVICE_CHECK) and skipped.  Used to predict a layer's
+ * remote experts from a look-ahead routing and to find those a prediction
+ * missed. */
+MOE_API moe_status moe_experts_touched(const int32_t *topk_idx, int64_t A, int32_t E,
+                               uint8_t *touched, cudaStream_t stream);
+
 /* Host-side poll of an event with a deadline: MOE_OK once it has completed,
  * MOE_ERR_TIMEOUT after timeout_ms milliseconds, MOE_ERR_CUDA on error. */
 MOE_API moe_status moe_wait_ready(cudaEvent_t ev, int32_t timeout_ms);

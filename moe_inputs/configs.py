@@ -102,7 +102,8 @@ CONFIGS: dict[int, MoEConfig] = {
 
 # Reduced cases of the same kernels for profiler captures, a few GB on the
 # device: the decode shape with 32 routed experts (about 4 tokens each, as in
-# the 128-token decode step), the prefill shape and the FP8 shape with 32 experts.
+# the 128-token decode step), the prefill shape and the FP8 shape with 32
+# experts; and a two-layer decode pipeline for the selective-fetch measurement.
 PROFILE_CASES: dict[int, MoEConfig] = {
     21: CONFIGS[2].with_(cfg_id=21, name="r1_decode_shape_E32_T16", T=16, E=32, local_count=8),
     # the 8K-prefill router (T, H, E as in the prefill workload) with small experts
@@ -111,6 +112,9 @@ PROFILE_CASES: dict[int, MoEConfig] = {
                          local_count=8),
     25: CONFIGS[5].with_(cfg_id=25, name="r1_fp8_shape_E32_T512", T=512, E=32, local_count=8,
                          layers=1),
+    # two decode-sized layers through the prefetch pipeline: 32 tokens touch about
+    # 60 % of the routed experts, the case a selective fetch is for
+    26: CONFIGS[2].with_(cfg_id=26, name="r1_decode_T32_2layers", T=32, layers=2),
 }
 
 

@@ -102,6 +102,9 @@ _SIGS = {
     "moe_prefetch_layer_paced": ([vp, vp, sz, sz, vp, vp, vp, ctypes.c_uint32,
                                   ctypes.POINTER(moe_progress), i32, vp], i32),
     "moe_pace_threshold": ([i64, i64, i32, ctypes.c_uint32, i32], ctypes.c_uint32),
+    "moe_prefetch_slots": ([vp, vp, sz, i32, ctypes.POINTER(i32), i32, vp, vp, vp,
+                            ctypes.c_uint32, vp], i32),
+    "moe_experts_touched": ([vp, i64, i32, vp, vp], i32),
     "moe_combine": ([i32, i32, i32, vp, vp, vp, i32, vp, i32, vp], i32),
     "moe_prefetch_layer": ([vp, vp, sz, sz, vp, vp, vp], i32),
     "moe_peer_fetch_plan": ([i32, i32, i64, i32, ctypes.POINTER(moe_peer_copy), i32,
@@ -157,6 +160,8 @@ moe_prefetch_layer_flagged = _lib.moe_prefetch_layer_flagged
 moe_grouped_ffn_paced = _lib.moe_grouped_ffn_paced
 moe_prefetch_layer_paced = _lib.moe_prefetch_layer_paced
 moe_pace_threshold = _lib.moe_pace_threshold
+moe_prefetch_slots = _lib.moe_prefetch_slots
+moe_experts_touched = _lib.moe_experts_touched
 moe_combine = _lib.moe_combine
 moe_prefetch_layer = _lib.moe_prefetch_layer
 moe_peer_fetch_plan = _lib.moe_peer_fetch_plan

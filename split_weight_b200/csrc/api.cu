@@ -320,6 +320,43 @@ moe_status moe_prefetch_layer_paced(const void* src, void* dst, size_t bytes, si
                         lead_chunks, ready_out);
 }
 
+moe_status moe_prefetch_slots(const void* src, void* dst, size_t slot_bytes, int32_t pool_slots,
+                              const int32_t* slots, int32_t n, cudaStream_t copy_stream,
+                              cudaEvent_t wait_free, uint32_t* flags, uint32_t epoch,
+                              cudaEvent_t ready_out) {
+    if (n < 0 || pool_slots < 0 || (n > 0 && (!src || !dst || !slots || slot_bytes == 0)) ||
+        !flags || !aligned(flags, 4))
+        return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_slots: n >= 0, pool_slots >= 0, buffers, "
+                    "slots, slot_bytes > 0 and 4-byte aligned flags needed");
+    for (int32_t i = 0; i < n; ++i)
+        if (slots[i] < 0 || slots[i] >= pool_slots)
+            return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_slots: slot %d outside [0, %d)",
+                        slots[i], pool_slots);
+    if (n > 0) {   // the pool images of src and dst may not overlap
+        const size_t span = (size_t)pool_slots * slot_bytes;
+        const char* s = static_cast<const char*>(src);
+        char* d = static_cast<char*>(dst);
+        if ((s < d + span) && (d < s + span))
+            return fail(MOE_ERR_INVALID_ARG, "moe_prefetch_slots: source and destination overlap");
+    }
+    if (wait_free) SWB_CUDA(cudaStreamWaitEvent(copy_stream, wait_free, 0));
+    for (int32_t i = 0; i < n;) {   // runs of consecutive slots: one copy each
+        int32_t j = i + 1;
+        while (j < n && slots[j] == slots[j - 1] + 1) ++j;
+        const size_t off = (size_t)slots[i] * slot_bytes;
+        SWB_CUDA(cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off,
+                                 (size_t)(j - i) * slot_bytes, cudaMemcpyDeviceToDevice,
+                                 copy_stream));
+        for (int32_t q = i; q < j; ++q) {
+            const moe_status st = stream_write_u32(copy_stream, flags + slots[q], epoch);
+            if (st != MOE_OK) return st;
+        }
+        i = j;
+    }
+    if (ready_out) SWB_CUDA(cudaEventRecord(ready_out, copy_stream));
+    return MOE_OK;
+}
+
 uint32_t moe_pace_threshold(int64_t chunk, int64_t n_chunks, int32_t lead_chunks, uint32_t base,
                             int32_t steps) {
     return swb::pace_threshold(chunk, n_chunks, lead_chunks, base, steps);

@@ -51,6 +51,17 @@ __global__ void __launch_bounds__(kThreads) k_hist(const int32_t* __restrict__ i
         blk_counts[(int64_t)blockIdx.x * E + e] = cnt[e];
 }
 
+// touched[e] = 1 for every expert some assignment selects (entries outside
+// [0, E) are reported and skipped, as in k_hist); the caller zeroed touched.
+__global__ void k_touched(const int32_t* __restrict__ idx, int64_t A, int E,
+                          uint8_t* __restrict__ touched, int* err) {
+    for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < A;
+         a += (int64_t)gridDim.x * blockDim.x) {
+        const int e = load_expert(idx, a, A, E, err);
+        if (e >= 0) touched[e] = 1;
+    }
+}
+
 // One block of 1024 threads: offsets[] and each block's first row per expert.
 __global__ void __launch_bounds__(1024) k_scan(const int32_t* __restrict__ blk_counts, int nb,
                                                int E, int32_t* __restrict__ blk_base,
@@ -263,6 +274,25 @@ size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E) {
     if (T < 0 || k <= 0 || E <= 0) return 0;
     const int64_t nb = num_blocks((int64_t)T * k);
     return (size_t)(2 * nb * E) * sizeof(int32_t);
+}
+
+moe_status moe_experts_touched(const int32_t* topk_idx, int64_t A, int32_t E, uint8_t* touched,
+                               cudaStream_t stream) {
+    if (A < 0 || E <= 0 || E > MOE_MAX_EXPERTS || !touched || (A > 0 && !topk_idx))
+        return fail(MOE_ERR_INVALID_ARG, "moe_experts_touched: A=%lld E=%d, touched and topk_idx "
+                    "needed", (long long)A, E);
+    int* err = nullptr;
+    moe_status st = device_error_word(&err);
+    if (st != MOE_OK) return st;
+    SWB_CUDA(cudaMemsetAsync(touched, 0, (size_t)E, stream));
+    if (A == 0) return MOE_OK;
+    int sms = 0;
+    if ((st = sm_count(&sms)) != MOE_OK) return st;
+    const int64_t want = (A + 255) / 256;
+    const unsigned g = (unsigned)(want < 4 * sms ? want : 4 * sms);
+    k_touched<<<g, 256, 0, stream>>>(topk_idx, A, E, touched, err);
+    SWB_LAUNCHED("moe_experts_touched");
+    return MOE_OK;
 }
 
 }  // extern "C"

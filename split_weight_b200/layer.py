@@ -267,6 +267,14 @@ class MoELayer:
         return self.y
 
 
+def remote_slots(pool_slot: np.ndarray, touched: np.ndarray) -> set[int]:
+    """Remote-pool slots of the experts marked in `touched` [E] (the
+    moe_experts_touched bytes), from the (pool << 31) | slot table."""
+    ps = np.asarray(pool_slot, dtype=np.int32).view(np.uint32)
+    sel = (np.asarray(touched[:len(ps)]) != 0) & ((ps >> 31) == 1)
+    return set(int(v) for v in (ps[sel] & 0x7FFFFFFF))
+
+
 class PrefetchPipeline:
     """Consecutive MoE layers whose remote experts are fetched ahead into two
     alternate buffers by moe_prefetch_layer on a copy-engine stream.
@@ -305,12 +313,25 @@ class PrefetchPipeline:
     stream for an even share of those reports (moe_prefetch_layer_paced).
     The copy then runs spread over the grouped GEMMs instead of as one burst
     beside them, and never waits for work enqueued after it.
+
+    With select=True (per-slot flags: gate_slots = 1) the fetch is selective:
+    execution g routes the next layer's tokens ahead of time with that
+    layer's router on its own input x (a look-ahead prediction), and right
+    after its grouped GEMM enqueues fetches only the remote slots so
+    predicted (moe_prefetch_slots); when execution g + 1 has routed for
+    real, the slots the prediction missed are fetched before its grouped
+    GEMM, which waits per slot.  Each execution costs one host
+    synchronisation (the touched-expert bytes of its routing and of the
+    prediction), and fetches (predicted ∪ missed) slots instead of all.
+    select_stats records, per execution, the touched, predicted and missed
+    slot counts.
     """
 
     def __init__(self, layers: list[MoELayer], peer_stores: list[torch.Tensor],
                  remote_bytes: int, device: torch.device | str = "cuda", chunk_bytes: int = 0,
                  split: bool = True, gate_slots: int = 0, window_block=None,
-                 gate_timeout_ns: int = 0, pace_steps: int = 0, pace_lead: int = 0):
+                 gate_timeout_ns: int = 0, pace_steps: int = 0, pace_lead: int = 0,
+                 select: bool = False):
         self.layers, self.peer_stores = layers, peer_stores
         self.remote_bytes, self.chunk_bytes = remote_bytes, chunk_bytes
         self.split, self.pending = split, None
@@ -328,15 +349,33 @@ class PrefetchPipeline:
         self.flags = None
         self.pace_steps, self.pace_lead, self.g_pace0 = 0, 0, 0
         self.progress_words = torch.zeros(3, dtype=torch.int32, device=dev)
-        self.configure(gate_slots=gate_slots, pace_steps=pace_steps, pace_lead=pace_lead)
+        self.select, self._pred = False, None
+        self.fetched = [set(), set()]
+        self.select_stats: list[dict] = []
+        self.configure(gate_slots=gate_slots, pace_steps=pace_steps, pace_lead=pace_lead,
+                       select=select)
 
     def configure(self, split: bool | None = None, gate_slots: int | None = None,
                   window_block=False, pace_steps: int | None = None,
-                  pace_lead: int | None = None) -> None:
+                  pace_lead: int | None = None, select: bool | None = None) -> None:
         """Switches the schedule between runs (after a synchronisation: no
         fetch may be in flight).  window_block=False leaves it as it is."""
         if split is not None:
             self.split = split
+        if select is not None:
+            self.select = select
+            self.fetched = [set(), set()]
+            if select and self._pred is None:
+                l0, dev = self.layers[0], self.device
+                T, k, E = l0.shape.T, l0.shape.k, l0.shape.E
+                self._pred = {
+                    "idx": torch.empty(max(T, 1), k, dtype=torch.int32, device=dev),
+                    "w": torch.empty(max(T, 1), k, dtype=torch.float32, device=dev),
+                    "ws": torch.empty_like(l0.route_ws),
+                    "touched": torch.zeros(2, E, dtype=torch.uint8, device=dev),
+                    "host": torch.zeros(2, E, dtype=torch.uint8).pin_memory(),
+                    "ev": torch.cuda.Event(),
+                }
         if pace_lead is not None:
             self.pace_lead = pace_lead
         if pace_steps is not None:
@@ -358,6 +397,9 @@ class PrefetchPipeline:
         if self.pace_steps > 0:
             assert self.gate_slots > 0 and self.pace_steps >= 2, \
                 "a paced fetch needs readiness flags and at least 2 steps"
+        if self.select:
+            assert self.gate_slots == 1 and self.pace_steps == 0, \
+                "a selective fetch needs per-slot flags (gate_slots=1) and no pacing"
         self.pending = None
 
     def progress(self, execution: int) -> Progress:
@@ -391,6 +433,16 @@ class PrefetchPipeline:
             L.check(L.moe_prefetch_layer(src, dst, hi - lo, self.chunk_bytes,
                                          self.copy_stream.cuda_stream, wf, rd))
 
+    def _fetch_slots(self, layer: int, buf: int, slots: list[int], wait_free, epoch: int) -> None:
+        """Selective fetch of the given remote slots of `layer` into bufs[buf]."""
+        n_slots = self.remote_bytes // self.stride
+        arr = (ctypes.c_int32 * max(len(slots), 1))(*slots)
+        wf = wait_free.cuda_event if wait_free is not None else None
+        L.check(L.moe_prefetch_slots(self.peer_stores[layer].data_ptr(), self.bufs[buf].data_ptr(),
+                                     self.stride, n_slots, arr, len(slots),
+                                     self.copy_stream.cuda_stream, wf, self.flags[buf].data_ptr(),
+                                     epoch & 0xFFFFFFFF, None))
+
     def _cut(self) -> int:
         if self.gate_slots > 0:
             chunk = self.gate_slots * self.stride
@@ -422,6 +474,9 @@ class PrefetchPipeline:
         n = len(self.layers)
         self.copy_stream.wait_stream(torch.cuda.current_stream(self.device))
         self.pending = None
+        if self.select:   # nothing predicted yet: the first execution fetches what it misses
+            self.fetched = [set(), set()]
+            return
         for i in range(1 if self.pace_steps > 0 else 2):
             self.prefetch((self.g + i) % n, (self.g + i) % 2, None, self.g + i)
 
@@ -436,6 +491,11 @@ class PrefetchPipeline:
             self.window_block(l, x, stream)
         layer.route(x, h)
         layer.permute(x, h)
+        if prefetch and self.select:
+            self._run_selective(l, x, stream, ffn_events, wrap)
+            layer.combine(h)
+            self.g += 1
+            return layer.y
         gate = None
         if prefetch and self.gate_slots > 0:
             gate = ReadyGate(self.flags[b], g + 1, self.gate_slots, self.gate_timeout_ns)
@@ -470,6 +530,51 @@ class PrefetchPipeline:
         layer.combine(h)
         self.g += 1
         return layer.y
+
+    def _run_selective(self, l: int, x: torch.Tensor, stream: torch.cuda.Stream, ffn_events,
+                       wrap: bool) -> None:
+        """Execution g of the selective schedule, after its routing and
+        permutation: the look-ahead prediction of the next layer, one host
+        synchronisation, the missed slots, the grouped GEMM, then the
+        predicted fetch of execution g + 1."""
+        n = len(self.layers)
+        layer, h, b, g = self.layers[l], stream.cuda_stream, self.g % 2, self.g
+        s, pr = layer.shape, self._pred
+        L.check(L.moe_experts_touched(layer.topk_idx.data_ptr(), s.T * s.k, s.E,
+                                      pr["touched"][0].data_ptr(), h))
+        nxt = (l + 1) % n
+        ahead = l + 1 < n or wrap
+        if ahead:   # the next layer's router on this layer's input
+            nl = self.layers[nxt]
+            L.check(L.moe_route(ctypes.byref(nl._cfg), x.data_ptr(), _DT[nl.shape.x_dtype],
+                                nl.w_gate.data_ptr(), _ptr(nl.bias), pr["idx"].data_ptr(),
+                                pr["w"].data_ptr(), pr["ws"].data_ptr(), pr["ws"].numel(), h))
+            L.check(L.moe_experts_touched(pr["idx"].data_ptr(), s.T * s.k, s.E,
+                                          pr["touched"][1].data_ptr(), h))
+        with torch.cuda.stream(stream):
+            pr["host"].copy_(pr["touched"], non_blocking=True)
+        pr["ev"].record(stream)
+        pr["ev"].synchronize()
+        touched = remote_slots(layer.weights.pool_slot, pr["host"][0].numpy())
+        missed = sorted(touched - self.fetched[b])
+        if missed:   # after the predicted fetch of this buffer on the copy stream
+            self._fetch_slots(l, b, missed, self.free[b], g + 1)
+            self.fetched[b] |= set(missed)
+        stats = {"touched": len(touched), "missed": len(missed)}
+        gate = ReadyGate(self.flags[b], g + 1, 1, self.gate_timeout_ns)
+        if ffn_events is not None:
+            ffn_events[0].record(stream)
+        layer.grouped_ffn(h, self.bufs[b], gate, x=x)
+        if ffn_events is not None:
+            ffn_events[1].record(stream)
+        self.free[b].record(stream)
+        if ahead:
+            nb = (g + 1) % 2
+            pred = sorted(remote_slots(self.layers[nxt].weights.pool_slot, pr["host"][1].numpy()))
+            self._fetch_slots(nxt, nb, pred, self.free[nb], g + 2)
+            self.fetched[nb] = set(pred)
+            stats["predicted_next"] = len(pred)
+        self.select_stats.append(stats)
 
     def run(self, xs: list[torch.Tensor], stream: torch.cuda.Stream | None = None,
             prefetch: bool = True, wrap: bool = True) -> list[torch.Tensor]:
