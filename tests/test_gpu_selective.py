@@ -87,7 +87,7 @@ def test_prefetch_slots_copies_only_the_listed_slots(cuda_device):
 @pytest.mark.parametrize("cfg,act", [(MID_SIGMOID, "bf16"), (MID_FP8, "bf16")],
                          ids=["bf16", "e4m3_weights"])
 def test_selective_pipeline_equals_resident_layers_and_oracle(cfg, act):
-    cfg = cfg.with_(cfg_id=cfg.cfg_id + 300, layers=3)
+    cfg = cfg.with_(cfg_id=cfg.cfg_id + 150, layers=3)
     dls = [mdev.build_layer(cfg, layer=l, act_dtype=act) for l in range(cfg.layers)]
     ref = []
     for d in dls:
