@@ -252,8 +252,13 @@ typedef struct moe_expert_table {
  *                        [I/128, rows] fp32 go to the workspace, which must
  *                        hold moe_grouped_ffn_workspace_size(d) bytes.
  *                        Requires H % 256 == 0.
- * x_perm_scales and the workspace are ignored (may be NULL, size 0) in the
- * two bf16-activation combinations.
+ * x_perm_scales is ignored (may be NULL) in the two bf16-activation
+ * combinations.  There the workspace is optional: with
+ * moe_grouped_ffn_workspace_size(d) bytes (16-byte aligned) the kernels
+ * take their tiles from two counters in it, each CTA the next tile when it
+ * is ready for one, which balances tiles of unequal size; with NULL (or
+ * fewer bytes) each CTA takes a fixed round-robin share.  The results are
+ * the same bits either way.  A workspace serves one call at a time.
  * Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.
  * ---------------------------------------------------------------------- */
 typedef struct moe_ffn_desc {

@@ -269,8 +269,11 @@ using namespace swb;
 extern "C" {
 
 size_t moe_grouped_ffn_workspace_size(const moe_ffn_desc* d) {
+    if (!d) return 0;
+    // bf16 activations: the two launches' tile counters (dynamic tile schedule)
+    if (d->act_dtype != MOE_E4M3) return kTileCounterBytes;
     // e4m3 activations: the fp32 scales of the e4m3 intermediate h, [I/128][rows]
-    if (!d || d->act_dtype != MOE_E4M3 || d->T <= 0 || d->k <= 0 || d->I <= 0) return 0;
+    if (d->T <= 0 || d->k <= 0 || d->I <= 0) return 0;
     const int64_t rows = (int64_t)d->T * d->k + (d->has_shared ? d->T : 0);
     return (size_t)((d->I / 128) * rows * 4 + 255) / 256 * 256;
 }
@@ -432,6 +435,13 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
             (st = stream_write_u32(stream, progress->tiles + 1, 0u)) != MOE_OK)
             return st;
     }
+    // bf16 activations with a workspace: the two launches take their tiles
+    // from counters in it (dynamic schedule); without one, round-robin
+    int32_t* tile_counters = nullptr;
+    if (!f8 && workspace && workspace_bytes >= kTileCounterBytes && aligned(workspace, 16)) {
+        tile_counters = static_cast<int32_t*>(workspace);
+        SWB_CUDA(cudaMemsetAsync(tile_counters, 0, 2 * sizeof(int32_t), stream));
+    }
     if (f8) return ffn_f8(d, tbl, lay, x_perm, x_perm_scales, h, y_perm,
                           static_cast<float*>(workspace), (int)rows, G, a, progress, stream);
 
@@ -465,6 +475,7 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     a.out = static_cast<__nv_bfloat16*>(h);
     a.ld_out = d->I;
     set_progress(a, progress, 0);
+    a.tile_counter = tile_counters;
     if ((st = launch_w<kGated>(w8, bn, a, (int)rows, G, stream)) != MOE_OK) return st;
 
     // GEMM2: y = h W_down^T
@@ -486,6 +497,7 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     a.out = static_cast<__nv_bfloat16*>(y_perm);
     a.ld_out = d->H;
     set_progress(a, progress, 1);
+    a.tile_counter = tile_counters ? tile_counters + 1 : nullptr;
     if (d->H % (2 * kBM) == 0) return launch_w<kPair>(w8, bn, a, (int)rows, G, stream);
     return launch_w<kSingle>(w8, bn, a, (int)rows, G, stream);
 }

@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ Tables tb;
+    __shared__ TileQueue tq;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t stages = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -86,6 +87,10 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&acc_full[a]), 1);
             mbar_init(smem_u32(&acc_empty[a]), C::kEpiWarps);
+        }
+        for (int q = 0; q < kTileRing; ++q) {   // consumers: MMA thread, epilogue and converter warps
+            mbar_init(smem_u32(&tq.full[q]), 1);
+            mbar_init(smem_u32(&tq.empty[q]), 1 + C::kEpiWarps + C::kConvWarps);
         }
         fence_mbar_init();
         if (p.gather) {
@@ -114,7 +119,9 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
             int stage = 0, passed = -1;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int it = 0; ok; ++it) {
+                const int tile = tile_produce(p, tq, it, abort_flag, p.err);
+                if (tile >= total) break;
                 const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
                 if (!gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)) break;
                 const CUtensorMap* wm = &p.w_map[t.map];
@@ -156,7 +163,11 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         int stage = 0, passed = -1;
         uint32_t phase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int it = 0; ok; ++it) {
+            int tile = 0;
+            if (lane == 0) tile = tile_produce(p, tq, it, abort_flag, p.err);
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            if (tile >= total) break;
             const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
             if (!__all_sync(0xffffffffu, lane != 0 || gate_wait(p, t.map, t.slot, passed, abort_flag, p.err)))
                 break;
@@ -217,7 +228,10 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_use[2] = {0u, 0u};
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int it = 0; ok; ++it) {
+                const int tile = tile_consume(p, tq, it, abort_flag, p.err);
+                if (tile >= total) break;
+                tile_release(p, tq, it);
                 const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
                 if (!mbar_wait(smem_u32(&acc_empty[acc]), (acc_use[acc] & 1u) ^ 1u, abort_flag,
                                p.err))
@@ -265,7 +279,11 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         int stage = 0, passed = -1;
         uint32_t phase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int it = 0; ok; ++it) {
+            const int tile = tile_consume(p, tq, it, abort_flag, p.err);
+            if (tile >= total) break;
+            __syncwarp();
+            if (lane == 0) tile_release(p, tq, it);
             const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
             // the block scales sit in the remote buffer too: read them only once
             // landed, and L2-coherently while a gated fetch may be writing other slots
@@ -337,7 +355,11 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         constexpr int kCols = BN / (C::kEpiWarps / 4);
         int acc = 0;
         uint32_t acc_use[2] = {0u, 0u};
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        for (int it = 0;; ++it) {
+            const int tile = tile_consume(p, tq, it, abort_flag, p.err);
+            if (tile >= total) break;
+            __syncwarp();
+            if (lane == 0) tile_release(p, tq, it);
             const Tile t = decode_tile<BN, C::kRowsPerTile>(tile, tb, G);
             bool ok = mbar_wait(smem_u32(&acc_full[acc]), acc_use[acc] & 1u, abort_flag, p.err);
             if (!__all_sync(0xffffffffu, ok)) break;

@@ -2,6 +2,8 @@
 // (per-expert token tiles, balanced and 16-aligned) and the SwiGLU helper.
 #pragma once
 
+#include <climits>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -69,6 +71,9 @@ struct alignas(64) FfnArgs {
     uint32_t* progress_tiles;
     uint32_t progress_base;
     int32_t progress_steps;
+    // dynamic tile schedule (NULL: static round-robin): the launch's next tile
+    // index, zeroed by the host before the launch
+    int32_t* tile_counter;
     // tile enumeration order: position i holds group order[i] (local experts
     // and the shared one first, then the remote experts in slot order, the
     // order in which a fetch fills them)
@@ -233,6 +238,49 @@ __device__ __forceinline__ void report_progress(const FfnArgs& p, int total) {
         if (old == cur) break;
         cur = old;
     }
+}
+
+// The tiles of one CTA, in the order all its roles take them.  Static
+// (tile_counter NULL): blockIdx.x, + gridDim.x, ...  Dynamic: the producer
+// takes the launch's next tile from a global counter whenever it is ready
+// for one, so a CTA that drew small tiles takes more of them, and hands each
+// index to the other roles through a ring in shared memory; an index >= the
+// tile count (or an abort) ends every role.
+constexpr int kTileRing = 4;
+// workspace bytes the bf16-activation call uses for its two tile counters
+constexpr size_t kTileCounterBytes = 256;
+
+struct TileQueue {
+    int id[kTileRing];
+    uint64_t full[kTileRing];    // one arrival: the producer wrote id[s]
+    uint64_t empty[kTileRing];   // one arrival per consumer role (warp or thread)
+};
+
+__device__ __forceinline__ int tile_produce(const FfnArgs& p, TileQueue& q, int it,
+                                            volatile int* abort, int* err) {
+    if (!p.tile_counter) return (int)blockIdx.x + it * (int)gridDim.x;
+    const int s = it % kTileRing;
+    const uint32_t ph = (uint32_t)(it / kTileRing) & 1u;
+    if (!mbar_wait(smem_u32(&q.empty[s]), ph ^ 1u, abort, err)) return INT_MAX;
+    const int t = *abort ? INT_MAX : atomicAdd(p.tile_counter, 1);
+    *reinterpret_cast<volatile int*>(&q.id[s]) = t;
+    mbar_arrive(smem_u32(&q.full[s]));
+    return t;
+}
+
+// Every thread of a consumer role reads the index; then one thread per role
+// calls tile_release for the same `it`.
+__device__ __forceinline__ int tile_consume(const FfnArgs& p, TileQueue& q, int it,
+                                            volatile int* abort, int* err) {
+    if (!p.tile_counter) return (int)blockIdx.x + it * (int)gridDim.x;
+    const int s = it % kTileRing;
+    const uint32_t ph = (uint32_t)(it / kTileRing) & 1u;
+    if (!mbar_wait(smem_u32(&q.full[s]), ph, abort, err)) return INT_MAX;
+    return *reinterpret_cast<volatile int*>(&q.id[s]);
+}
+
+__device__ __forceinline__ void tile_release(const FfnArgs& p, TileQueue& q, int it) {
+    if (p.tile_counter) mbar_arrive(smem_u32(&q.empty[it % kTileRing]));
 }
 
 // Two fp32 values rounded to bf16 (round to nearest even), lo in bits 0-15.

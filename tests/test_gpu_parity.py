@@ -4,6 +4,7 @@ Routing indices, counts, offsets and the permutation must be bit-exact; the
 sigmoid routing weights too (their arithmetic is defined in fp32).  Layer
 outputs must satisfy max|err| <= 2e-2 * max|ref| (bf16 path).
 """
+import ctypes
 import gc
 
 import numpy as np
@@ -166,6 +167,26 @@ def test_pool_invariance_bit_identical(seed):
         dl = mdev.build_layer(cfg, placement=pl)
         y = run_layer(dl).y
         assert torch.equal(y, y_ref), f"placement {pl} changed the output"
+
+
+@pytest.mark.parametrize("cfg,act", [(MID_SIGMOID, "bf16"), (MID_BN256, "bf16"),
+                                     (MID_BN128_FP8, "bf16")],
+                         ids=["bf16", "bf16_bn256", "e4m3_weights"])
+def test_dynamic_and_static_tile_schedules_bit_identical(cfg, act):
+    """With a workspace the grouped GEMM's CTAs take tiles from a counter
+    (dynamic schedule); without one, a fixed round-robin share.  Every output
+    element is computed by one tile in a fixed order, so the bits agree."""
+    dl = mdev.build_layer(cfg, act_dtype=act)
+    y_dyn = run_layer(dl).y.clone()
+    ml, h = dl.layer, torch.cuda.current_stream().cuda_stream
+    assert ml.ffn_ws.numel() >= L.moe_grouped_ffn_workspace_size(ctypes.byref(ml._desc)) >= 256
+    tbl = ml.weights.table()
+    L.check(L.moe_grouped_ffn(ctypes.byref(ml._desc), ctypes.byref(tbl), ml.x_perm.data_ptr(),
+                              None, ml.offsets.data_ptr(), ml.h.data_ptr(), ml.y_perm.data_ptr(),
+                              None, 0, h))
+    ml.combine(h)
+    sync_check()
+    assert torch.equal(ml.y, y_dyn)
 
 
 def test_all_tokens_one_expert_is_dense_ffn():
