@@ -389,8 +389,12 @@ def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
     nocopy_ms = e0.elapsed_time(e1) / reps
     ffn_nocopy = sum(a.elapsed_time(b) for st in ffn_ev for a, b in st) / reps
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the baseline every schedule is measured against: the whole remote buffer of
+    # one layer as one copy (the schedule's own chunking and flags excluded)
+    from split_weight_b200 import _lib as L
     c0.record(pipe.copy_stream)
-    pipe.prefetch(0, 0, None)
+    L.check(L.moe_prefetch_layer(pipe.peer_stores[0].data_ptr(), pipe.bufs[0].data_ptr(),
+                                 pipe.remote_bytes, 0, pipe.copy_stream.cuda_stream, None, None))
     c1.record(pipe.copy_stream)
     torch.cuda.synchronize()
     copy_ms = c0.elapsed_time(c1)
@@ -400,7 +404,9 @@ def prefetch_overlap(cfg, pipe, step, stream, piped_ms, steps):
     torch.cuda.synchronize()
     exposed = max(0.0, (piped_ms - nocopy_ms) / cfg.layers)
     return {
-        "schedule": ((f"paced by the grouped GEMM's progress ({pipe.pace_steps} steps, "
+        "schedule": (("selective: predicted remote slots after the grouped GEMM, missed ones "
+                      "before the next" if pipe.select else
+                      f"paced by the grouped GEMM's progress ({pipe.pace_steps} steps, "
                       f"{pipe.pace_lead} chunks ahead)" if pipe.pace_steps else
                       "halves between grouped GEMMs" if pipe.split else "whole, after the grouped GEMM")
                      + (f"; readiness flags every {pipe.gate_slots} slots" if pipe.gate_slots else
