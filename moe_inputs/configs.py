@@ -114,7 +114,7 @@ PROFILE_CASES: dict[int, MoEConfig] = {
                          layers=1),
     # two decode-sized layers through the prefetch pipeline: 32 tokens touch about
     # 60 % of the routed experts, the case a selective fetch is for
-    26: CONFIGS[2].with_(cfg_id=26, name="r1_decode_T32_2layers", T=32, layers=2),
+    33: CONFIGS[2].with_(cfg_id=33, name="r1_decode_T32_2layers", T=32, layers=2),
 }
 
 

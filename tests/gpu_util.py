@@ -38,6 +38,9 @@ MID_BN256_H384 = config(2).with_(cfg_id=31, name="mid_bn256_T2048_H384_I256_E8_k
 MID_BN256_FP8 = config(5).with_(cfg_id=28, name="mid_bn256_fp8_T2048_H512_I256_E8_k1", T=2048,
                                 H=512, I=256, E=8, k=1, n_group=1, topk_group=1, local_count=3,
                                 layers=1)
+# e4m3 weights with H = 384: the down GEMM runs single 128-row tiles
+MID_FP8_H384 = config(5).with_(cfg_id=32, name="mid_fp8_T300_H384_I256_E32", T=300, H=384, I=256,
+                               E=32, k=4, n_group=4, topk_group=2, local_count=8, layers=1)
 MID_BN128 = config(2).with_(cfg_id=29, name="mid_bn128_T1000_H384_I256_E16_k2", T=1000, H=384,
                             I=256, E=16, k=2, n_group=4, topk_group=2, local_count=5)
 MID_BN128_FP8 = config(5).with_(cfg_id=30, name="mid_bn128_fp8_T1000_H512_I256_E16_k2", T=1000,

@@ -17,8 +17,8 @@ from oracle import workload as ow
 from split_weight_b200 import _lib as L
 
 from gpu_util import (DECODE_FP8, MAX_EXPERTS, MID_BN128, MID_BN128_FP8, MID_BN256, MID_BN256_FP8,
-                      MID_BN256_H384,
-                      MID_FP8, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN, RTOL_BF16, RTOL_FP8,
+                      MID_BN256_H384, MID_FP8, MID_FP8_H384, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN,
+                      RTOL_BF16, RTOL_FP8,
                       SPARSE_DECODE, assert_close_rel, run_layer, sync_check, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -80,7 +80,8 @@ def test_small_layer_full_parity(cfg):
     assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
 
 
-@pytest.mark.parametrize("cfg", [MID_BN256, MID_BN256_H384, MID_BN256_FP8, MID_BN128, MID_BN128_FP8],
+@pytest.mark.parametrize("cfg", [MID_BN256, MID_BN256_H384, MID_BN256_FP8, MID_BN128, MID_BN128_FP8,
+                                 MID_FP8_H384],
                          ids=lambda c: c.name)
 def test_mid_layer_each_tile_width_full_parity(cfg):
     """Whole mid-size layers whose experts get ~256 or ~125 tokens each, so
