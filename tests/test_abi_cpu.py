@@ -157,3 +157,50 @@ def test_injected_cuda_failure_is_reported_and_cleared():
     assert rc == L.MOE_ERR_CUDA
     assert "injected" in L.moe_last_error()
     L.moe_debug_fail_next_cuda_calls(0)
+
+
+@pytest.mark.parametrize("n,lead,base,steps", [(24, 2, 100, 24), (24, 0, 0, 24), (6, 2, 100, 4),
+                                               (5, 9, 7, 3), (192, 3, 0xFFFFFFF0, 24),
+                                               (3, 0, 5, 40)])
+def test_pace_threshold_spreads_chunks_over_the_reports(n, lead, base, steps):
+    """moe_pace_threshold: the first `lead` chunks need nothing beyond base;
+    the others need a share of the reports that never decreases along the
+    fetch and stays within base + steps (wrap-around arithmetic)."""
+    t = [L.moe_pace_threshold(c, n, lead, base & 0xFFFFFFFF, steps) for c in range(n)]
+    rel = [(v - base) & 0xFFFFFFFF for v in t]
+    assert all(r == 0 for r in rel[:lead])
+    assert all(a <= b for a, b in zip(rel, rel[1:]))
+    assert all(0 <= r <= steps for r in rel)
+    if lead < n:
+        assert rel[-1] == ((n - lead) * (steps + 1)) // (n - lead + 1)
+
+
+def test_paced_and_selective_calls_check_arguments_first():
+    """Argument errors come back before anything is enqueued (no GPU here)."""
+    p = 1 << 12
+    pr = L.moe_progress(p, p + 4, 0, 8)
+    bad_steps = L.moe_progress(p, p + 4, 0, 1)
+    odd_word = L.moe_progress(p + 2, p + 4, 0, 8)
+    assert L.moe_prefetch_layer_paced(p, 1 << 24, 1 << 20, 1 << 16, None, None, p, 1, None, 0,
+                                      None) == L.MOE_ERR_INVALID_ARG            # no pace
+    assert L.moe_prefetch_layer_paced(p, 1 << 24, 1 << 20, 1 << 16, None, None, p, 1,
+                                      ctypes.byref(odd_word), 0, None) == L.MOE_ERR_INVALID_ARG
+    assert L.moe_prefetch_layer_paced(p, 1 << 24, 1 << 20, 1 << 16, None, None, p, 1,
+                                      ctypes.byref(pr), -1, None) == L.MOE_ERR_INVALID_ARG
+    assert L.moe_prefetch_layer_paced(p, 1 << 24, 1 << 20, 0, None, None, p, 1,
+                                      ctypes.byref(pr), 0, None) == L.MOE_ERR_INVALID_ARG
+    d, tbl = _ffn(), _table([0, 1, 1 << 31, (1 << 31) | 1])
+    assert L.moe_grouped_ffn_paced(ctypes.byref(d), ctypes.byref(tbl), None, None, p, None, None,
+                                   None, p, p, p, None, 0, None) == L.MOE_ERR_INVALID_ARG
+    assert L.moe_grouped_ffn_paced(ctypes.byref(d), ctypes.byref(tbl), None, ctypes.byref(bad_steps),
+                                   p, None, None, None, p, p, p, None, 0,
+                                   None) == L.MOE_ERR_INVALID_ARG
+    slots = (ctypes.c_int32 * 3)(0, 4, 9)
+    assert L.moe_prefetch_slots(p, 1 << 24, 256, 9, slots, 3, None, None, p, 1,
+                                None) == L.MOE_ERR_INVALID_ARG              # slot 9 of 9
+    assert L.moe_prefetch_slots(p, p + 256, 256, 9, slots, 2, None, None, p, 1,
+                                None) == L.MOE_ERR_INVALID_ARG              # overlapping pools
+    assert L.moe_prefetch_slots(p, 1 << 24, 256, 9, slots, -1, None, None, p, 1,
+                                None) == L.MOE_ERR_INVALID_ARG
+    assert L.moe_experts_touched(p, 10, 0, p, None) == L.MOE_ERR_INVALID_ARG
+    assert L.moe_experts_touched(None, 10, 8, p, None) == L.MOE_ERR_INVALID_ARG

@@ -135,3 +135,31 @@ def test_paced_pipeline_equals_resident_layers_and_oracle(cfg, act):
                              f"pass {rep} layer {l} against the oracle")
     # every execution's call ended: the word sits at the next execution's base
     assert _u32(pipe.progress_words)[0] == pipe.progress(pipe.g).base
+
+
+def test_paced_call_ends_the_word_when_it_has_no_work_or_fails(cuda_device):
+    """The call's final write of the progress word comes whatever the call did:
+    with no tokens, and after an argument error (here H not a multiple of
+    128), so that a fetch paced by it is never left waiting."""
+    dl = mdev.build_layer(MID_SIGMOID)
+    ml = dl.layer
+    words = torch.zeros(3, dtype=torch.int32, device="cuda")
+    h = torch.cuda.current_stream().cuda_stream
+    tbl = ml.weights.table()
+    empty = L.moe_ffn_desc(0, ml._desc.H, ml._desc.I, ml._desc.E, ml._desc.k, ml._desc.w_dtype,
+                           ml._desc.act_dtype, ml._desc.has_shared)
+    pr = Progress(words, 40, 6).c_struct()
+    assert L.moe_grouped_ffn_paced(ctypes.byref(empty), ctypes.byref(tbl), None, ctypes.byref(pr),
+                                   None, None, None, None, ml.offsets.data_ptr(), None, None,
+                                   None, 0, h) == L.MOE_OK
+    sync_check()
+    assert _u32(words)[0] == 40 + 6 + 1
+    bad = L.moe_ffn_desc(ml._desc.T, 100, ml._desc.I, ml._desc.E, ml._desc.k, ml._desc.w_dtype,
+                         ml._desc.act_dtype, ml._desc.has_shared)
+    pr = Progress(words, 80, 6).c_struct()
+    assert L.moe_grouped_ffn_paced(ctypes.byref(bad), ctypes.byref(tbl), None, ctypes.byref(pr),
+                                   ml.x_perm.data_ptr(), None, None, None, ml.offsets.data_ptr(),
+                                   ml.h.data_ptr(), ml.y_perm.data_ptr(), None, 0,
+                                   h) == L.MOE_ERR_INVALID_ARG
+    sync_check()
+    assert _u32(words)[0] == 80 + 6 + 1
