@@ -234,18 +234,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
     return d;
 }
 
-// The same for 64-byte rows in the 64-byte swizzle (8-row groups 512 bytes
-// apart, layout type 4).
-__device__ __forceinline__ uint64_t sw64_desc(uint32_t smem_addr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(1u) << 16;
-    d |= static_cast<uint64_t>(512u >> 4) << 32;
-    d |= static_cast<uint64_t>(1u) << 46;
-    d |= static_cast<uint64_t>(4u) << 61;
-    return d;
-}
-
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
 // 4-5 = 1), A and B bf16 (bits 7-9, 10-12 = 1), both K-major, N >> 3 at
 // bits 17-22, M >> 4 at bits 24-28.

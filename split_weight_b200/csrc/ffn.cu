@@ -12,6 +12,8 @@
 //   warp 0      TMA producer (one thread): weight tile(s) + token rows
 //   warp 1      tcgen05.mma issuer (one thread); owns the TMEM allocation
 //   warps 2..   epilogue (4, 8 or 16 warps): TMEM -> registers -> (SwiGLU) -> bf16
+//   then        e4m3 weights only: 8 converter warps, staged e4m3 codes x block
+//               scale -> the bf16 operand buffers the MMA reads
 // The MMA puts weight rows on M (128 per instruction) and the expert's tokens
 // on N (16..256), so a decode-sized expert with 4 tokens costs an N=16 MMA,
 // not a 128-row tile.  A CTA holds one or two weight tiles per stage:
@@ -93,32 +95,33 @@ moe_status launch_w(bool w8, int bn, const FfnArgs& a, int rows, int G, cudaStre
     return w8 ? launch_bn<MODE, true>(bn, a, rows, G, s) : launch_bn<MODE, false>(bn, a, rows, G, s);
 }
 
-// Token tile from the mean tokens per routed expert, 16..256.
-int pick_bn(int64_t A, int E) {
+// Token tile from the mean tokens per routed expert, 16..256.  e4m3 weights
+// are converted once per token tile, so they move to 256-token tiles sooner:
+// routing skew leaves the experts a token picks with more than the mean, and
+// a 256-token tile converts an expert's weights once where 128-token tiles
+// convert them twice.
+int pick_bn(int64_t A, int E, bool w8 = false) {
     const int64_t mean = (A + E - 1) / E;
     if (mean <= 8) return 16;
     if (mean <= 16) return 32;
     if (mean <= 32) return 64;
-    if (mean <= 160) return 128;
+    if (mean <= (w8 ? 96 : 160)) return 128;
     return 256;
 }
 
 // 3-D map {K, rows, slot} over one pool of expert images.  bf16 weights are
-// loaded straight into the MMA operand layout (bks = 64: 128-byte rows and
-// swizzle; bks = 32: 64-byte rows and swizzle); e4m3 weights as plain
-// bks-byte rows for the converter warps.  The e4m3 map for the tensor-core
-// fp8 path (f8mma) loads 128-byte rows straight into the MMA operand layout.
+// loaded straight into the MMA operand layout (64-wide boxes: 128-byte rows
+// and swizzle); e4m3 weights as plain 64-byte rows for the converter warps.
+// The e4m3 map for the tensor-core fp8 path (f8mma) loads 128-byte rows
+// straight into the MMA operand layout.
 moe_status encode_weight_map(CUtensorMap* m, const void* base, int64_t offset, int32_t count,
-                             int64_t stride, int32_t K, int32_t rows, bool w8, bool f8mma = false,
-                             int bks = kBK) {
+                             int64_t stride, int32_t K, int32_t rows, bool w8, bool f8mma = false) {
     const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)count};
     const uint64_t strides[2] = {(uint64_t)K * (w8 ? 1 : 2), (uint64_t)stride};
-    const uint32_t box[3] = {(uint32_t)(f8mma ? 128 : bks), (uint32_t)kBM, 1u};
+    const uint32_t box[3] = {(uint32_t)(f8mma ? 128 : kBK), (uint32_t)kBM, 1u};
     return encode_tiled(m, w8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                         const_cast<char*>(static_cast<const char*>(base)) + offset, dims, strides,
-                        box, (w8 && !f8mma) ? CU_TENSOR_MAP_SWIZZLE_NONE
-                             : (!f8mma && bks == 32) ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                     : CU_TENSOR_MAP_SWIZZLE_128B);
+                        box, (w8 && !f8mma) ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 moe_status encode_act_map8(CUtensorMap* m, const void* base, int64_t rows, int32_t K,
@@ -130,14 +133,14 @@ moe_status encode_act_map8(CUtensorMap* m, const void* base, int64_t rows, int32
                         strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// bf16 rows {K, rows}: boxes of bks (64: 128-byte swizzle; 32: 64-byte) x box_rows.
+// bf16 rows {K, rows}: boxes of 64 (128-byte swizzle) x box_rows.
 moe_status encode_act_map(CUtensorMap* m, const void* base, int64_t rows, int32_t K,
-                          uint32_t box_rows, int bks = kBK) {
+                          uint32_t box_rows) {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
     const uint64_t strides[1] = {(uint64_t)K * 2};
-    const uint32_t box[2] = {(uint32_t)bks, box_rows};
+    const uint32_t box[2] = {(uint32_t)kBK, box_rows};
     return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                        strides, box, bks == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+                        strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 moe_status validate(const moe_ffn_desc* d, const moe_expert_table* tb, moe_expert_layout* lay) {
@@ -421,9 +424,8 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     const void* base[2] = {tbl->local_base, tbl->remote_base};
     const int32_t count[2] = {tbl->local_count, tbl->remote_count};
     const int64_t stride[2] = {tbl->local_stride, tbl->remote_stride};
-    const int bn = pick_bn(A, d->E);
     const bool w8 = d->w_dtype == MOE_E4M3;
-    const int bks = stage_k(bn, w8);   // K per stage of the kernel launched (Cfg::kBKs)
+    const int bn = pick_bn(A, d->E, w8);
     a.w_base[0] = static_cast<const uint8_t*>(tbl->local_base);
     a.w_base[1] = static_cast<const uint8_t*>(tbl->remote_base);
     a.w_base[2] = static_cast<const uint8_t*>(tbl->shared);
@@ -448,26 +450,25 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     // GEMM1: h = silu(X W_gate^T) * (X W_up^T)
     for (int q = 0; q < 2; ++q)
         if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.gu_offset, count[q],
-                                                    stride[q], d->H, 2 * d->I, w8, false, bks)) != MOE_OK)
+                                                    stride[q], d->H, 2 * d->I, w8)) != MOE_OK)
             return st;
     if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.gu_offset, 1,
-                                                 lay.bytes, d->H, 2 * d->I, w8, false, bks)) != MOE_OK)
+                                                 lay.bytes, d->H, 2 * d->I, w8)) != MOE_OK)
         return st;
     a.scale_off = lay.gu_scale_offset;
     a.kblocks = d->H / 128;
     if (perm_src) {   // token tiles gathered from x [T, H] through perm_src
         const uint64_t dims[2] = {(uint64_t)d->H, (uint64_t)d->T};
         const uint64_t strides[1] = {(uint64_t)d->H * 2};
-        const uint32_t box[2] = {(uint32_t)bks, 1u};
+        const uint32_t box[2] = {(uint32_t)kBK, 1u};
         if ((st = encode_tiled(&a.x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x_perm),
-                               dims, strides, box,
-                               bks == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) != MOE_OK)
+                               dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != MOE_OK)
             return st;
         a.perm_src = perm_src;
         a.gather = 1;
     } else {
-        if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H, kBoxN, bks)) != MOE_OK) return st;
-        if ((st = encode_act_map(&a.act_map64, x_perm, rows, d->H, 64, bks)) != MOE_OK) return st;
+        if ((st = encode_act_map(&a.act_map, x_perm, rows, d->H, kBoxN)) != MOE_OK) return st;
+        if ((st = encode_act_map(&a.act_map64, x_perm, rows, d->H, 64)) != MOE_OK) return st;
     }
     a.K = d->H;
     a.M = d->I;
@@ -481,16 +482,16 @@ moe_status ffn_run(const moe_ffn_desc* d, const moe_expert_table* tbl, const moe
     // GEMM2: y = h W_down^T
     for (int q = 0; q < 2; ++q)
         if (count[q] > 0 && (st = encode_weight_map(&a.w_map[q], base[q], lay.down_offset,
-                                                    count[q], stride[q], d->I, d->H, w8, false, bks)) != MOE_OK)
+                                                    count[q], stride[q], d->I, d->H, w8)) != MOE_OK)
             return st;
     if (d->has_shared && (st = encode_weight_map(&a.w_map[2], tbl->shared, lay.down_offset, 1,
-                                                 lay.bytes, d->I, d->H, w8, false, bks)) != MOE_OK)
+                                                 lay.bytes, d->I, d->H, w8)) != MOE_OK)
         return st;
     a.scale_off = lay.down_scale_offset;
     a.kblocks = d->I / 128;
     a.gather = 0;
-    if ((st = encode_act_map(&a.act_map, h, rows, d->I, kBoxN, bks)) != MOE_OK) return st;
-    if ((st = encode_act_map(&a.act_map64, h, rows, d->I, 64, bks)) != MOE_OK) return st;
+    if ((st = encode_act_map(&a.act_map, h, rows, d->I, kBoxN)) != MOE_OK) return st;
+    if ((st = encode_act_map(&a.act_map64, h, rows, d->I, 64)) != MOE_OK) return st;
     a.K = d->I;
     a.M = d->H;
     a.up_row = 0;

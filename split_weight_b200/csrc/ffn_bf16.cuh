@@ -9,20 +9,29 @@ namespace {
 
 constexpr int kConvThreads = 256;              // e4m3 -> bf16 converter warps (8)
 
-// Per stage: the bf16 weight tile(s) the MMA reads (128-byte swizzled), the
-// token tile, and for e4m3 weights the staging tile(s) TMA writes.
+// bf16 weights: one ring of stages, each the bf16 weight tile(s) the MMA
+// reads (128-byte swizzled) and the token tile.  e4m3 weights: a TMA ring of
+// {token tile, e4m3 staging tile(s)} and a ring of kStagesY converted bf16
+// weight operands, so that the token tile of a 256-token tile and three TMA
+// stages fit beside the two operand buffers the converters and the MMA
+// alternate on.
 template <int BN, int MODE, bool W8>
 struct Cfg {
     static constexpr int kNA = MODE == kSingle ? 1 : 2;           // weight tiles per stage
-    static constexpr int kBKs = stage_k(BN, W8);                  // K per stage
-    static constexpr bool kSw64 = kBKs == 32;
+    static constexpr int kBKs = kBK;                              // K per stage
     static constexpr uint32_t kATile = kBM * kBKs * 2;            // one bf16 weight tile
     static constexpr uint32_t kA8Tile = kBM * kBKs;               // one e4m3 tile as loaded
     static constexpr uint32_t kAStage = kATile * kNA;
     static constexpr uint32_t kBStage = BN * kBKs * 2;
     static constexpr uint32_t kA8Stage = W8 ? kA8Tile * kNA : 0;
-    static constexpr uint32_t kStageBytes = kAStage + kBStage + kA8Stage;
-    static constexpr int kStages = (kSmemBudget / kStageBytes) > 12 ? 12 : (kSmemBudget / kStageBytes);
+    static constexpr int kStagesY = W8 ? 2 : 0;                   // converted operand buffers
+    // offsets within a TMA stage: bf16 weights | tokens, or tokens | e4m3 codes
+    static constexpr uint32_t kTokOff = W8 ? 0 : kAStage;
+    static constexpr uint32_t kCodeOff = kBStage;
+    static constexpr uint32_t kStageBytes = W8 ? kBStage + kA8Stage : kAStage + kBStage;
+    static constexpr uint32_t kRingBudget = W8 ? kSmemBudgetW8 - kStagesY * kAStage : kSmemBudget;
+    static constexpr int kStages = (kRingBudget / kStageBytes) > 12 ? 12 : (kRingBudget / kStageBytes);
+    static constexpr uint32_t kYOff = kStages * kStageBytes;      // the operand ring, after the TMA ring
     static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
     static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
     static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
@@ -32,10 +41,11 @@ struct Cfg {
     static constexpr int kConvFirstWarp = 2 + kEpiWarps;
     static constexpr int kThreads = 64 + 32 * (kEpiWarps + kConvWarps);
     static constexpr int kRowsPerTile = MODE == kPair ? 2 * kBM : kBM;  // output features
-    static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + 1024;
+    static constexpr size_t kDynSmem = (size_t)kStages * kStageBytes + kStagesY * kAStage + 1024;
     static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                   "TMEM allocation must be a power of two in [32, 512]");
-    static_assert(kStages >= 2, "pipeline needs two stages");
+    static_assert(kStages >= (W8 ? 3 : 2), "pipeline needs two stages (three beside the converters)");
+    static_assert(kStageBytes % 1024 == 0 && kAStage % 1024 == 0, "operand tiles sit on 1024-byte swizzle atoms");
 };
 // 16 e4m3 weights (one 16-byte chunk of a staged row) times their block
 // scale, rounded to bf16: 32 bytes, the two 16-byte chunks that follow.
@@ -63,7 +73,8 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     using C = Cfg<BN, MODE, W8>;
     extern __shared__ uint8_t dyn_smem[];
     __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
-    __shared__ __align__(8) uint64_t conv_bar[W8 ? C::kStages : 1];  // bf16 tiles converted
+    __shared__ __align__(8) uint64_t conv_bar[W8 ? C::kStagesY : 1];  // operand buffer converted
+    __shared__ __align__(8) uint64_t yempty_bar[W8 ? C::kStagesY : 1]; // operand buffer read by the MMAs
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -82,7 +93,10 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&empty_bar[s]), 1);
-            if constexpr (W8) mbar_init(smem_u32(&conv_bar[s]), C::kConvWarps);
+        }
+        for (int y = 0; y < C::kStagesY; ++y) {
+            mbar_init(smem_u32(&conv_bar[y]), C::kConvWarps);
+            mbar_init(smem_u32(&yempty_bar[y]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&acc_full[a]), 1);
@@ -136,11 +150,11 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                     const uint32_t sa = stages + stage * C::kStageBytes;
                     mbar_arrive_expect_tx(fb, tx);
                     // e4m3 weights land in the staging area, bf16 ones straight in the operand
-                    const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
+                    const uint32_t sw = W8 ? sa + C::kCodeOff : sa;
                     const uint32_t w_step = W8 ? C::kA8Tile : C::kATile;
                     tma_load_3d(sw, wm, fb, kb * C::kBKs, t.m0, t.slot);
                     if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * C::kBKs, row_a1, t.slot);
-                    const uint32_t sb = sa + C::kAStage;
+                    const uint32_t sb = sa + C::kTokOff;
                     int r = 0;
                     for (; r + 64 <= t.n_mma; r += 64)
                         tma_load_2d(sb + r * C::kBKs * 2, &p.act_map64, fb, kb * C::kBKs, t.row0 + r);
@@ -200,10 +214,10 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                     break;
                 }
                 const uint32_t sa = stages + stage * C::kStageBytes;
-                const uint32_t sb = sa + C::kAStage;
+                const uint32_t sb = sa + C::kTokOff;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(fb, tx);
-                    const uint32_t sw = W8 ? sa + C::kAStage + C::kBStage : sa;
+                    const uint32_t sw = W8 ? sa + C::kCodeOff : sa;
                     const uint32_t w_step = W8 ? C::kA8Tile : C::kATile;
                     tma_load_3d(sw, wm, fb, kb * C::kBKs, t.m0, t.slot);
                     if constexpr (C::kNA == 2) tma_load_3d(sw + w_step, wm, fb, kb * C::kBKs, row_a1, t.slot);
@@ -225,8 +239,8 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int stage = 0, acc = 0;
-            uint32_t phase = 0, acc_use[2] = {0u, 0u};
+            int stage = 0, acc = 0, ys = 0;
+            uint32_t phase = 0, yphase = 0, acc_use[2] = {0u, 0u};
             bool ok = true;
             for (int it = 0; ok; ++it) {
                 const int tile = tile_consume(p, tq, it, abort_flag, p.err);
@@ -240,24 +254,37 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
                 const uint32_t idesc = idesc_bf16_f32(kBM, t.n_mma);
                 for (int kb = 0; kb < KB; ++kb) {
-                    const uint32_t ready_bar = W8 ? smem_u32(&conv_bar[stage]) : smem_u32(&full_bar[stage]);
-                    if (!mbar_wait(ready_bar, phase, abort_flag, p.err)) {
+                    // e4m3 weights: the converters have filled operand buffer ys
+                    // (after this stage's TMA landed)
+                    if (W8 && !mbar_wait(smem_u32(&conv_bar[ys]), yphase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = stages + stage * C::kStageBytes;
-                    const uint32_t sb = sa + C::kAStage;
+                    const uint32_t sb = stages + stage * C::kStageBytes + C::kTokOff;
+                    const uint32_t sa = W8 ? stages + C::kYOff + ys * C::kAStage
+                                           : stages + stage * C::kStageBytes;
 #pragma unroll
                     for (int kk = 0; kk < C::kBKs / 16; ++kk) {
                         const uint32_t accum = (kb | kk) != 0;
-                        const uint64_t bd = C::kSw64 ? sw64_desc(sb + kk * 32) : sw128_desc(sb + kk * 32);
+                        const uint64_t bd = sw128_desc(sb + kk * 32);
                         const uint32_t a0 = sa + kk * 32, a1 = a0 + C::kATile;
-                        mma_bf16_ss(d0, C::kSw64 ? sw64_desc(a0) : sw128_desc(a0), bd, idesc, accum);
+                        mma_bf16_ss(d0, sw128_desc(a0), bd, idesc, accum);
                         if constexpr (C::kNA == 2)
-                            mma_bf16_ss(d0 + BN, C::kSw64 ? sw64_desc(a1) : sw128_desc(a1), bd, idesc, accum);
+                            mma_bf16_ss(d0 + BN, sw128_desc(a1), bd, idesc, accum);
                     }
                     mma_commit(smem_u32(&empty_bar[stage]));
+                    if constexpr (W8) {
+                        mma_commit(smem_u32(&yempty_bar[ys]));
+                        if (++ys == C::kStagesY) {
+                            ys = 0;
+                            yphase ^= 1u;
+                        }
+                    }
                     if (++stage == C::kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -276,8 +303,8 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
         // row is 2 kBKs bytes in the matching swizzle.  One 128x128 block scale
         // covers the whole stage (kBKs columns of K, 128 rows).
         const int ct = threadIdx.x - 32 * C::kConvFirstWarp;  // 0 .. kConvThreads-1
-        int stage = 0, passed = -1;
-        uint32_t phase = 0;
+        int stage = 0, ys = 0, passed = -1;
+        uint32_t phase = 0, yphase = 0;
         bool ok = true;
         for (int it = 0; ok; ++it) {
             const int tile = tile_consume(p, tq, it, abort_flag, p.err);
@@ -306,13 +333,16 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                     s0n = scale(sc0, kb + 1);
                     if constexpr (C::kNA == 2) s1n = scale(sc1, kb + 1);
                 }
-                ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err);
+                // the stage's codes have landed, and the MMAs are done with the
+                // operand buffer's previous contents
+                ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.err) &&
+                     mbar_wait(smem_u32(&yempty_bar[ys]), yphase ^ 1u, abort_flag, p.err);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
                 }
-                const uint32_t sa = stages + stage * C::kStageBytes;
-                const uint32_t s8 = sa + C::kAStage + C::kBStage;
+                const uint32_t sa = stages + C::kYOff + ys * C::kAStage;
+                const uint32_t s8 = stages + stage * C::kStageBytes + C::kCodeOff;
 #pragma unroll
                 for (int a = 0; a < C::kNA; ++a) {
                     const float sc = a == 0 ? s0 : s1;
@@ -326,9 +356,9 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                                      : "r"(s8 + a * C::kA8Tile + r * C::kBKs + c * 16));
                         e4m3x16_to_bf16(in, sc, lo, hi);
                         // the operand row r (kBKs * 2 bytes): 16-byte chunk j at
-                        // j ^ (r % 8) (128-byte swizzle) or j ^ ((r / 2) % 4) (64-byte)
+                        // j ^ (r % 8) (128-byte swizzle)
                         const uint32_t row = sa + a * C::kATile + r * (C::kBKs * 2);
-                        const uint32_t sw = C::kSw64 ? ((r >> 1) & 3) : (r & 7);
+                        const uint32_t sw = r & 7;
                         const uint32_t j0 = (2 * c) ^ sw, j1 = (2 * c + 1) ^ sw;
                         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + j0 * 16),
                                      "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w)
@@ -341,7 +371,11 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
                 // generic-proxy stores -> visible to the tensor core's async proxy
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&conv_bar[stage]));
+                if (lane == 0) mbar_arrive(smem_u32(&conv_bar[ys]));
+                if (++ys == C::kStagesY) {
+                    ys = 0;
+                    yphase ^= 1u;
+                }
                 if (++stage == C::kStages) {
                     stage = 0;
                     phase ^= 1u;

@@ -21,12 +21,7 @@ constexpr int kBoxN = 16;                      // token rows per TMA box
 constexpr uint32_t kABytes = kBM * kBK * 2;    // one weight tile, 16 KB
 constexpr uint32_t kSmemBudget = 200 * 1024;   // pipeline stages
 
-// K per pipeline stage of the bf16-operand kernel (kind::f16): 64 (128-byte
-// operand rows, 128-byte swizzle), or 32 (64-byte rows, 64-byte swizzle) for
-// e4m3 weights at 256-token tiles, where a 64-wide stage with its e4m3 staging
-// would leave room for two stages only.  The host encodes its tensor maps'
-// boxes with the same value.
-__host__ __device__ constexpr int stage_k(int bn, bool w8) { return (w8 && bn >= 256) ? 32 : kBK; }
+constexpr uint32_t kSmemBudgetW8 = 208 * 1024; // both rings, e4m3 weights on bf16 MMAs
 
 struct alignas(64) FfnArgs {
     CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}

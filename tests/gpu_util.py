@@ -43,9 +43,15 @@ MID_FP8_H384 = config(5).with_(cfg_id=32, name="mid_fp8_T300_H384_I256_E32", T=3
                                E=32, k=4, n_group=4, topk_group=2, local_count=8, layers=1)
 MID_BN128 = config(2).with_(cfg_id=29, name="mid_bn128_T1000_H384_I256_E16_k2", T=1000, H=384,
                             I=256, E=16, k=2, n_group=4, topk_group=2, local_count=5)
-MID_BN128_FP8 = config(5).with_(cfg_id=30, name="mid_bn128_fp8_T1000_H512_I256_E16_k2", T=1000,
+# e4m3 weights take 256-token tiles from ~97 tokens per expert on (they are
+# converted once per token tile): ~88 tokens per expert keeps 128-token tiles,
+# ~125 reaches 256-token tiles holding ragged row counts
+MID_BN128_FP8 = config(5).with_(cfg_id=30, name="mid_bn128_fp8_T700_H512_I256_E16_k2", T=700,
                                 H=512, I=256, E=16, k=2, n_group=4, topk_group=2, local_count=5,
                                 layers=1)
+MID_BN256_FP8_K2 = config(5).with_(cfg_id=34, name="mid_bn256_fp8_T1000_H512_I256_E16_k2", T=1000,
+                                   H=512, I=256, E=16, k=2, n_group=4, topk_group=2, local_count=5,
+                                   layers=1)
 # the largest shapes the ABI takes: 1024 experts, k = 32, 32 groups (one per lane)
 MAX_EXPERTS = config(2).with_(cfg_id=26, name="max_E1024_k32_G32_T64", T=64, H=256, I=128,
                               E=1024, k=32, n_group=32, topk_group=4, local_count=256)
@@ -80,3 +86,14 @@ def run_layer(dl: mdev.DeviceLayer):
     dl.layer.forward(dl.x)
     sync_check()
     return dl.layer
+
+
+def tile_width(cfg) -> int:
+    """Token-tile width the grouped GEMM picks for a layer from its mean
+    tokens per routed expert (the library's rule, restated to check that a
+    test reaches the width it is written for)."""
+    mean = -(-cfg.A // cfg.E)
+    for bn, top in ((16, 8), (32, 16), (64, 32), (128, 96 if cfg.w_dtype == "e4m3" else 160)):
+        if mean <= top:
+            return bn
+    return 256

@@ -17,6 +17,7 @@ from oracle import workload as ow
 from split_weight_b200 import _lib as L
 
 from gpu_util import (DECODE_FP8, MAX_EXPERTS, MID_BN128, MID_BN128_FP8, MID_BN256, MID_BN256_FP8,
+                      MID_BN256_FP8_K2, tile_width,
                       MID_BN256_H384, MID_FP8, MID_FP8_H384, MID_SIGMOID, MID_SOFTMAX, ONE_TOKEN,
                       RTOL_BF16, RTOL_FP8,
                       SPARSE_DECODE, assert_close_rel, run_layer, sync_check, to_np)
@@ -80,14 +81,16 @@ def test_small_layer_full_parity(cfg):
     assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
 
 
-@pytest.mark.parametrize("cfg", [MID_BN256, MID_BN256_H384, MID_BN256_FP8, MID_BN128, MID_BN128_FP8,
-                                 MID_FP8_H384],
-                         ids=lambda c: c.name)
-def test_mid_layer_each_tile_width_full_parity(cfg):
-    """Whole mid-size layers whose experts get ~256 or ~125 tokens each, so
-    the grouped GEMMs run 256-token tiles (one 512-column TMEM accumulator
-    set, the wide epilogue) or 128-token tiles with ragged row counts, in the
-    two-tile (gate/up, paired down) and single-tile (H = 384) down modes;
+@pytest.mark.parametrize("cfg,bn", [(MID_BN256, 256), (MID_BN256_H384, 256), (MID_BN256_FP8, 256),
+                                    (MID_BN256_FP8_K2, 256), (MID_BN128, 128), (MID_BN128_FP8, 128),
+                                    (MID_FP8_H384, 128)],
+                         ids=lambda c: getattr(c, "name", str(c)))
+def test_mid_layer_each_tile_width_full_parity(cfg, bn):
+    """Whole mid-size layers whose experts get enough tokens each for the
+    grouped GEMMs to run 256-token tiles (one 512-column TMEM accumulator
+    set, the wide epilogue; with e4m3 weights the converted-operand ring
+    beside three TMA stages) or 128-token tiles with ragged row counts, in
+    the two-tile (gate/up, paired down) and single-tile (H = 384) down modes;
     every output element against the oracle."""
     dl = mdev.build_layer(cfg)
     run_layer(dl)
@@ -95,13 +98,13 @@ def test_mid_layer_each_tile_width_full_parity(cfg):
     _check_routing(dl, idx_ref, w_ref)
     _check_permutation(dl, idx_ref)
     counts = np.diff(dl.layer.offsets.cpu().numpy())
-    mean = -(-cfg.A // cfg.E)
-    assert (mean > 160) if cfg.k == 1 else (32 < mean <= 160), "tile width not reached"
+    assert tile_width(cfg) == bn, "tile width not reached"
     assert (counts % 16 != 0).any(), "no ragged token tile"
     assert_close_rel(to_np(dl.layer.y[:cfg.T]), y_ref, _rtol(cfg), f"{cfg.name} y")
 
 
-@pytest.mark.parametrize("cfg", [MID_SIGMOID, MID_BN256, MID_BN128_FP8, SPARSE_DECODE],
+@pytest.mark.parametrize("cfg", [MID_SIGMOID, MID_BN256, MID_BN128_FP8, MID_BN256_FP8_K2,
+                                 SPARSE_DECODE],
                          ids=lambda c: c.name)
 def test_gathered_path_full_parity(cfg):
     """The grouped GEMM gathering its token rows itself from x through
@@ -171,8 +174,8 @@ def test_pool_invariance_bit_identical(seed):
 
 
 @pytest.mark.parametrize("cfg,act", [(MID_SIGMOID, "bf16"), (MID_BN256, "bf16"),
-                                     (MID_BN128_FP8, "bf16")],
-                         ids=["bf16", "bf16_bn256", "e4m3_weights"])
+                                     (MID_BN128_FP8, "bf16"), (MID_BN256_FP8_K2, "bf16")],
+                         ids=["bf16", "bf16_bn256", "e4m3_weights", "e4m3_weights_bn256"])
 def test_dynamic_and_static_tile_schedules_bit_identical(cfg, act):
     """With a workspace the grouped GEMM's CTAs take tiles from a counter
     (dynamic schedule); without one, a fixed round-robin share.  Every output
