@@ -287,7 +287,12 @@ MOE_API moe_status moe_grouped_ffn(const moe_ffn_desc *d, const moe_expert_table
  * outputs are undefined and moe_check_device() reports MOE_ERR_TIMEOUT.
  * flags: device, n_flags words, 4-byte aligned, written only by the copy
  * stream.  A NULL gate (or moe_grouped_ffn) reads the remote pool as it is:
- * the caller orders the fetch before the call (e.g. with the ready event). */
+ * the caller orders the fetch before the call (e.g. with the ready event).
+ * The waiting CTAs (one per SM) must leave room on their SMs for the fetch:
+ * between two buffers of one GPU cudaMemcpyAsync runs as a copy kernel on
+ * the SMs.  A gated call whose kernel would hold more than 55,296 registers
+ * per SM (the most measured to leave the copy running) returns MOE_ERR_CUDA
+ * instead of launching it; every kernel of this library is within it. */
 typedef struct moe_ready_gate {
     const uint32_t *flags;
     uint32_t epoch;

@@ -27,6 +27,8 @@
 // the next tile's main loop; the widest tiles (2 x 256 columns) use all 512
 // TMEM columns in one buffer and 16 epilogue warps, so the epilogue that
 // holds up the next tile's MMA is short.
+#include <atomic>
+
 #include "ffn_bf16.cuh"
 #include "ffn_f8.cuh"
 
@@ -34,6 +36,28 @@ namespace swb {
 namespace {
 
 // ---------------------------------------------------------------- host side
+// A call gated by readiness flags keeps its CTAs waiting for a fetch that may
+// run as a copy kernel on the same SMs: refuse a kernel whose CTA would leave
+// it less room than measured to work (kGatedRegsPerSm), rather than let the
+// gate's wait run out.
+// regs: the kernel's register count once looked up (-1 before), one per kernel.
+template <typename Kern>
+moe_status check_gated_room(const FfnArgs& a, Kern kern, std::atomic<int>& regs, int threads,
+                            const char* what) {
+    if (!a.ready_flags) return MOE_OK;
+    int r = regs.load(std::memory_order_relaxed);
+    if (r < 0) {
+        cudaFuncAttributes fa;
+        SWB_CUDA(cudaFuncGetAttributes(&fa, kern));
+        r = fa.numRegs;
+        regs.store(r, std::memory_order_relaxed);
+    }
+    if ((int64_t)r * threads > kGatedRegsPerSm)
+        return fail(MOE_ERR_CUDA, "%s: %d registers x %d threads leave a gated fetch's copy no room",
+                    what, r, threads);
+    return MOE_OK;
+}
+
 template <int BN, int MODE, bool W8>
 moe_status launch(const FfnArgs& a, int rows, int G, cudaStream_t s) {
     using C = Cfg<BN, MODE, W8>;
@@ -45,6 +69,8 @@ moe_status launch(const FfnArgs& a, int rows, int G, cudaStream_t s) {
     const int grid = (int)(bound < sms ? bound : sms);
     if (grid <= 0) return MOE_OK;
     auto kern = k_grouped_ffn<BN, MODE, W8>;
+    static std::atomic<int> regs{-1};
+    if ((st = check_gated_room(a, kern, regs, C::kThreads, "moe_grouped_ffn")) != MOE_OK) return st;
     SWB_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)C::kDynSmem));
     kern<<<grid, C::kThreads, C::kDynSmem, s>>>(a);
@@ -74,6 +100,8 @@ moe_status launch_f8(const FfnArgs& a, int rows, int G, cudaStream_t s) {
     const int grid = (int)(bound < sms ? bound : sms);
     if (grid <= 0) return MOE_OK;
     auto kern = k_grouped_ffn_f8<BN, MODE>;
+    static std::atomic<int> regs{-1};
+    if ((st = check_gated_room(a, kern, regs, C::kThreads, "moe_grouped_ffn (fp8)")) != MOE_OK) return st;
     SWB_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)C::kDynSmem));
     kern<<<grid, C::kThreads, C::kDynSmem, s>>>(a);

@@ -404,10 +404,12 @@ __global__ void __launch_bounds__(Cfg<BN, MODE, W8>::kThreads, 1)
             const int c_begin = part * kCols, c_end = min(t.n_rows, c_begin + kCols);
             constexpr int kChunks = kCols / 16;
             constexpr int kOut = (C::kNA == 2 && MODE != kGated) ? 2 : 1;
-            if constexpr (C::kAccBufs == 1 && !W8) {
+            if constexpr (C::kAccBufs == 1 && (!W8 || MODE == kGated)) {
                 // One accumulator set: the next tile's MMAs wait for it.  Pull this
                 // warp's columns out of TMEM into packed bf16 registers (at most 64),
-                // free the accumulator, then store while the MMAs run.
+                // free the accumulator, then store while the MMAs run.  With e4m3
+                // weights (8 epilogue warps, 128 columns each) only the gate/up
+                // launch does so: the paired down launch would hold 128.
                 uint32_t pk[kChunks][kOut][8];
 #pragma unroll
                 for (int ch = 0; ch < kChunks; ++ch) {

@@ -20,8 +20,15 @@ constexpr int kBK = 64;                        // K per stage: one 128-byte swiz
 constexpr int kBoxN = 16;                      // token rows per TMA box
 constexpr uint32_t kABytes = kBM * kBK * 2;    // one weight tile, 16 KB
 constexpr uint32_t kSmemBudget = 200 * 1024;   // pipeline stages
-
 constexpr uint32_t kSmemBudgetW8 = 208 * 1024; // both rings, e4m3 weights on bf16 MMAs
+
+// Registers a call gated by readiness flags may take on each SM (one CTA per
+// SM).  Its CTAs wait for a fetch; between two buffers of one GPU that fetch
+// (cudaMemcpyAsync) runs as a copy kernel on the SMs, so the CTA must leave
+// it room.  Measured on B200: a CTA holding 55,296 of the SM's 65,536
+// registers left the copy running beside it; one holding 59,904 kept it from
+// starting until the CTA ended, and the gated call's bounded wait ran out.
+constexpr int64_t kGatedRegsPerSm = 55296;
 
 struct alignas(64) FfnArgs {
     CUtensorMap w_map[3];      // 0 local pool, 1 remote pool, 2 shared expert: {K, rows, slot}
