@@ -535,6 +535,11 @@ MOE_API moe_status moe_check_device(void);
  * failure (MOE_ERR_CUDA) without being issued.  0 disarms it. */
 MOE_API void moe_debug_fail_next_cuda_calls(int32_t count);
 
+/* Test hook: a gated grouped-FFN launch (moe_ready_gate) is refused with
+ * MOE_ERR_CUDA when its kernel would hold more than `limit` registers per SM.
+ * 0 (or less) restores the library's limit, 55,296. */
+MOE_API void moe_debug_gated_regs_per_sm(int64_t limit);
+
 #ifdef __cplusplus
 }
 #endif

@@ -118,6 +118,7 @@ _SIGS = {
     "moe_wait_ready": ([vp, i32], i32),
     "moe_check_device": ([], i32),
     "moe_debug_fail_next_cuda_calls": ([i32], None),
+    "moe_debug_gated_regs_per_sm": ([i64], None),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -173,6 +174,7 @@ moe_pool_close = _lib.moe_pool_close
 moe_wait_ready = _lib.moe_wait_ready
 moe_check_device = _lib.moe_check_device
 moe_debug_fail_next_cuda_calls = _lib.moe_debug_fail_next_cuda_calls
+moe_debug_gated_regs_per_sm = _lib.moe_debug_gated_regs_per_sm
 
 
 def expert_layout(H: int, I: int, w_dtype: int) -> moe_expert_layout:

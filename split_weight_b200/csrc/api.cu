@@ -14,6 +14,7 @@ namespace swb {
 namespace {
 thread_local char g_last_error[512] = "";
 std::atomic<int> g_fail_next{0};
+std::atomic<int64_t> g_gated_regs{0};   // 0: the library's limit
 
 // One error word per device, in device memory owned by this library's
 // module (a __device__ variable: the library still allocates nothing).
@@ -37,6 +38,8 @@ moe_status fail(moe_status s, const char* fmt, ...) {
     va_end(ap);
     return s;
 }
+
+int64_t gated_regs_override() { return g_gated_regs.load(); }
 
 bool cuda_injected_failure() {
     int n = g_fail_next.load();
@@ -229,6 +232,7 @@ int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 void moe_debug_fail_next_cuda_calls(int32_t count) { g_fail_next.store(count > 0 ? count : 0); }
+void moe_debug_gated_regs_per_sm(int64_t limit) { g_gated_regs.store(limit > 0 ? limit : 0); }
 
 moe_status moe_expert_layout_get(int32_t H, int32_t I, moe_dtype w_dtype, moe_expert_layout* out) {
     if (!out) return fail(MOE_ERR_INVALID_ARG, "moe_expert_layout_get: out is NULL");

@@ -52,7 +52,8 @@ moe_status check_gated_room(const FfnArgs& a, Kern kern, std::atomic<int>& regs,
         r = fa.numRegs;
         regs.store(r, std::memory_order_relaxed);
     }
-    if ((int64_t)r * threads > kGatedRegsPerSm)
+    const int64_t limit = gated_regs_override() > 0 ? gated_regs_override() : kGatedRegsPerSm;
+    if ((int64_t)r * threads > limit)
         return fail(MOE_ERR_CUDA, "%s: %d registers x %d threads leave a gated fetch's copy no room",
                     what, r, threads);
     return MOE_OK;

@@ -20,6 +20,10 @@ moe_status fail(moe_status s, const char* fmt, ...);
 bool cuda_injected_failure();
 moe_status cuda_check(cudaError_t e, const char* what);
 
+// The registers per SM a gated launch may take, as set by the test hook
+// moe_debug_gated_regs_per_sm (0: the library's own limit).
+int64_t gated_regs_override();
+
 #define SWB_CUDA(call)                                                          \
     do {                                                                        \
         if (::swb::cuda_injected_failure())                                     \

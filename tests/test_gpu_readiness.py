@@ -55,6 +55,37 @@ def test_gate_with_flags_landed_equals_ungated(cfg, act):
 
 
 @pytest.mark.parametrize("cfg,act", CASES, ids=IDS)
+def test_gated_launch_without_room_for_the_copy_is_refused(cfg, act):
+    """A gated call's CTAs wait for a fetch that, between buffers of one GPU,
+    runs as a copy kernel on the same SMs.  With the register limit lowered
+    through the test hook the gated call is refused before its kernel is
+    launched, an ungated call still runs, and with the limit restored the
+    gated call gives the ungated bits."""
+    dl = mdev.build_layer(cfg, act_dtype=act)
+    y_ref = run_layer(dl).y.clone()
+    ml = dl.layer
+    flags = torch.full((5,), 7, dtype=torch.int32, device="cuda")
+    gate = ReadyGate(flags, 7, slots_per_flag=(cfg.E - cfg.local_count + 4) // 5)
+    h = torch.cuda.current_stream().cuda_stream
+    ml.route(dl.x, h)
+    ml.permute(dl.x, h)
+    launches = L.moe_kernel_launches()
+    L.moe_debug_gated_regs_per_sm(4096)
+    try:
+        with pytest.raises(L.MoEError) as err:
+            ml.grouped_ffn(h, None, gate, x=dl.x)
+        assert err.value.status == L.MOE_ERR_CUDA and "no room" in str(err.value)
+        assert L.moe_kernel_launches() == launches
+        ml.grouped_ffn(h, None, None, x=dl.x)     # no gate: no limit
+    finally:
+        L.moe_debug_gated_regs_per_sm(0)
+    ml.grouped_ffn(h, None, gate, x=dl.x)
+    ml.combine(h)
+    sync_check()
+    assert torch.equal(ml.y, y_ref)
+
+
+@pytest.mark.parametrize("cfg,act", CASES, ids=IDS)
 @pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
 def test_flag_gated_pipeline_equals_resident_layers_and_oracle(cfg, act, split):
     """Three layers through the alternate buffers with the compute stream
