@@ -164,7 +164,12 @@ constexpr int kBigT = 64, kBigE = 128, kBigK = 16;
 constexpr int kBigLd = kBigE + 4;  // row stride of the running sums in shared memory
 constexpr size_t kBigDynSmem = (size_t)kBigT * kBigLd * sizeof(float);
 
-template <typename XT>
+//
+// SPLIT: the z index of the grid is the 256-wide chunk.  The block computes
+// that chunk's sums alone and writes them to plane z of out ([chunks][T][E]);
+// k_reduce_parts then adds the planes in chunk order.  The same arithmetic,
+// spread over H/256 times as many blocks, so that every SM holds three.
+template <typename XT, bool SPLIT>
 __global__ void __launch_bounds__(128, 3) k_logits_big(const XT* __restrict__ x,
                                                        const float* __restrict__ wg, int T, int H,
                                                        int E, float* __restrict__ out) {
@@ -222,13 +227,14 @@ __global__ void __launch_bounds__(128, 3) k_logits_big(const XT* __restrict__ x,
     for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int q = 0; q < 4; ++q) p[i][q] = 0;
-    const int nk = H / kBigK;
-    load(0);
+    const int h_begin = SPLIT ? blockIdx.z * kChunk : 0;
+    const int nk = SPLIT ? (min(H - h_begin, kChunk)) / kBigK : H / kBigK;
+    load(h_begin);
     store(0);
     __syncthreads();
     for (int kt = 0; kt < nk; ++kt) {
         const int buf = kt & 1;
-        if (kt + 1 < nk) load((kt + 1) * kBigK);
+        if (kt + 1 < nk) load(h_begin + (kt + 1) * kBigK);
 #pragma unroll
         for (int kk = 0; kk < kBigK; ++kk) {
             const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][kk][ty * 4]);
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(128, 3) k_logits_big(const XT* __restrict__ x,
             }
         }
         const int h_next = (kt + 1) * kBigK;
-        if (h_next % kChunk == 0 || h_next >= H) {
+        if (!SPLIT && (h_next % kChunk == 0 || h_next >= H)) {
             const bool first = (h_next - 1) / kChunk == 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -263,14 +269,30 @@ __global__ void __launch_bounds__(128, 3) k_logits_big(const XT* __restrict__ x,
         if (kt + 1 < nk) store(buf ^ 1);
         __syncthreads();
     }
+    if constexpr (SPLIT) {
+        float* o = out + (int64_t)blockIdx.z * T * E;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int t = t0 + row_of(i);
-        if (t >= T) continue;
+        for (int i = 0; i < 8; ++i) {
+            const int t = t0 + row_of(i);
+            if (t >= T) continue;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = e0 + col_of(j);
-            if (e < E) out[(int64_t)t * E + e] = ls[row_of(i) * kBigLd + col_of(j)];
+            for (int q = 0; q < 4; ++q) {
+                const float2 v = unpack2(p[i][q]);
+                const int e = e0 + col_of(2 * q);   // col_of(2q + 1) = e + 1
+                if (e < E) o[(int64_t)t * E + e] = v.x;
+                if (e + 1 < E) o[(int64_t)t * E + e + 1] = v.y;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = t0 + row_of(i);
+            if (t >= T) continue;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int e = e0 + col_of(j);
+                if (e < E) out[(int64_t)t * E + e] = ls[row_of(i) * kBigLd + col_of(j)];
+            }
         }
     }
 }
@@ -483,14 +505,16 @@ struct RoutePlan {
 
 // Small batches split the h chunks over the grid (partial sums added in
 // chunk order by k_reduce_parts); large ones use the 64 x 128 tile when it
-// fills the GPU.
+// fills the GPU, with the chunks split over the grid as well (one block per
+// tile and chunk: a tile per block alone leaves two of an SM's three block
+// slots or fewer in use).
 RoutePlan plan(const moe_route_cfg* c) {
     RoutePlan p;
     const int64_t tiles32 = (int64_t)((c->T + 31) / 32) * ((c->E + 31) / 32);
     const int64_t tiles_big = (int64_t)((c->T + kBigT - 1) / kBigT) * ((c->E + kBigE - 1) / kBigE);
     const bool small = tiles32 < 512;
     p.tm = small ? 2 : (tiles_big >= 240 ? 8 : 4);
-    p.nsplit = small ? (c->H + kChunk - 1) / kChunk : 1;
+    p.nsplit = (small || p.tm == 8) ? (c->H + kChunk - 1) / kChunk : 1;
     return p;
 }
 
@@ -522,11 +546,14 @@ void launch_logits(const moe_route_cfg* c, const RoutePlan& p, const XT* x, cons
                    float* out, cudaStream_t s) {
     const int B = 16 * p.tm;
     dim3 grid((c->E + B - 1) / B, (c->T + B - 1) / B, p.nsplit);
-    if (p.tm == 8) {
+    if (p.tm == 8 && p.nsplit > 1) {
+        dim3 g((c->E + kBigE - 1) / kBigE, (c->T + kBigT - 1) / kBigT, p.nsplit);
+        k_logits_big<XT, true><<<g, 128, 0, s>>>(x, wg, c->T, c->H, c->E, out);
+    } else if (p.tm == 8) {
         dim3 g((c->E + kBigE - 1) / kBigE, (c->T + kBigT - 1) / kBigT);
-        cudaFuncSetAttribute(k_logits_big<XT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(k_logits_big<XT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kBigDynSmem);
-        k_logits_big<XT><<<g, 128, kBigDynSmem, s>>>(x, wg, c->T, c->H, c->E, out);
+        k_logits_big<XT, false><<<g, 128, kBigDynSmem, s>>>(x, wg, c->T, c->H, c->E, out);
     } else if (p.tm == 2) {
         k_logits<XT, 2, 2><<<grid, 256, 0, s>>>(x, wg, c->T, c->H, c->E, p.nsplit > 1, out);
     } else {

@@ -364,14 +364,18 @@ BIG_ROUTE_BF16 = config(2).with_(cfg_id=18, name="route_T7700_H512_E256", T=7700
 BIG_ROUTE_F32 = config(1).with_(cfg_id=19, name="route_f32_T20000_H256_E8", T=20000)
 MED_ROUTE = config(2).with_(cfg_id=22, name="route_T3001_H512_E256", T=3001, H=512, I=128)
 SPLIT_ROUTE = config(2).with_(cfg_id=20, name="route_T40_H7168_E256", T=40, I=128)
+# large batch with a last chunk of 128 h (H = 384): the chunk-split large tile
+BIG_ROUTE_H384 = config(2).with_(cfg_id=35, name="route_T7700_H384_E256", T=7700, H=384, I=128)
 
 
-@pytest.mark.parametrize("cfg", [BIG_ROUTE_BF16, BIG_ROUTE_F32, MED_ROUTE, SPLIT_ROUTE],
+@pytest.mark.parametrize("cfg", [BIG_ROUTE_BF16, BIG_ROUTE_F32, BIG_ROUTE_H384, MED_ROUTE,
+                                 SPLIT_ROUTE],
                          ids=lambda c: c.name)
 def test_routing_bit_exact_all_router_kernels(cfg, cuda_device):
-    """The three logits kernels (chunk-split for small batches, 64x64 and
-    128x128 tiles for large ones, ragged token counts) give the oracle's
-    bits; so do the selection and the permutation that follow."""
+    """The logits kernels (chunk-split small tiles for small batches, 64x64
+    tiles for medium ones, chunk-split 64x128 tiles for large ones, ragged
+    token counts and a short last chunk) give the oracle's bits; so do the
+    selection and the permutation that follow."""
     from moe_inputs.gen import layer_inputs
     from split_weight_b200 import MoELayer, SplitWeights
     li = layer_inputs(cfg)
