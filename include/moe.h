@@ -121,6 +121,11 @@ typedef struct moe_route_cfg {
     int32_t renormalize; /* see above */
 } moe_route_cfg;
 
+/* Workspace of moe_route (device, 16-byte aligned): the fp32 logits [T, E],
+ * or, when the logits kernel splits the h chunks over its grid (small and
+ * large batches), one [T, E] plane per 256-wide chunk, ceil(H/256) planes,
+ * summed in chunk order by the call (about 235 MB at T = 8192, H = 7168,
+ * E = 256).  0 for an invalid cfg. */
 MOE_API size_t moe_route_workspace_size(const moe_route_cfg *cfg);
 MOE_API moe_status moe_route(const moe_route_cfg *cfg, const void *x, moe_dtype x_dtype,
                      const float *w_gate, const float *bias, int32_t *topk_idx, float *topk_w,
