@@ -58,6 +58,34 @@ def test_route_rejects_bad_config(kw, code):
     assert L.moe_last_error()
 
 
+@pytest.mark.parametrize("T,H,planes", [
+    (128, 7168, 28),     # decode: small tiles split over the 28 chunks of 256 h
+    (3001, 512, 1),      # medium batch: 64x64 tiles, logits written once
+    (8192, 7168, 28),    # 8K prefill: 64x128 tiles split over the chunks
+    (7700, 384, 2),      # large batch with a short last chunk (256 + 128 h)
+])
+def test_route_workspace_holds_one_plane_per_split_chunk(T, H, planes):
+    """moe_route's workspace is one fp32 [T, E] plane per 256-wide chunk when
+    the logits kernel splits the chunks over its grid, else the logits alone
+    (host-side query, no GPU)."""
+    c = _route_cfg(T=T, H=H, E=256, k=8, score=L.MOE_SCORE_SIGMOID, n_group=8, topk_group=4)
+    assert L.moe_route_workspace_size(ctypes.byref(c)) == planes * T * 256 * 4
+
+
+@pytest.mark.parametrize("w,act,has_shared,want", [
+    (L.MOE_BF16, L.MOE_BF16, 1, 256),                 # two tile counters
+    (L.MOE_E4M3, L.MOE_BF16, 1, 256),                 # conversion path: the same counters
+    (L.MOE_E4M3, L.MOE_E4M3, 1, (2048 // 128) * (4096 * 8 + 4096) * 4),   # h's scales
+    (L.MOE_E4M3, L.MOE_E4M3, 0, (2048 // 128) * (4096 * 8) * 4),
+])
+def test_grouped_ffn_workspace_size(w, act, has_shared, want):
+    """bf16 activations: 256 bytes for the dynamic tile schedule's counters;
+    e4m3 activations: the fp32 scales of h, [I/128][rows], rounded up to 256
+    bytes (host-side query, no GPU)."""
+    d = L.moe_ffn_desc(4096, 7168, 2048, 256, 8, w, act, has_shared)
+    assert L.moe_grouped_ffn_workspace_size(ctypes.byref(d)) == -(-want // 256) * 256
+
+
 def test_route_rejects_null_misaligned_and_small_workspace():
     c = _route_cfg()
     assert L.moe_route(ctypes.byref(c), None, L.MOE_BF16, 16, None, 16, 16, None, 0,
