@@ -23,6 +23,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -119,11 +120,17 @@ def tensor_peak(peaks, mma_kind: str, timed_s: float):
     return 2.0 * bf16, f"fp8 dense taken as 2 x bf16 {which} (nominal ratio)"
 
 
+_COMMENTS = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
 def kernel_source_hash(files) -> str:
+    """Hash of the kernel sources with comments and blank space taken out: a
+    capture stays valid across an edit of the comments, not of the code."""
     h = hashlib.sha256()
     for name in files:
-        with open(os.path.join(ROOT, "split_weight_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "split_weight_b200", "csrc", name), encoding="utf-8") as f:
+            code = " ".join(_COMMENTS.sub(" ", f.read()).split())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

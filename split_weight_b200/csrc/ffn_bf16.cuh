@@ -1,5 +1,6 @@
 // The bf16 tensor-core grouped FFN kernel (kind::f16), with bf16 weights or
-// with e4m3 weights that converter warps dequantise into the staged tiles.
+// with e4m3 weights that converter warps dequantise into bf16 operand
+// buffers of their own.
 #pragma once
 
 #include "ffn_common.cuh"
@@ -35,7 +36,8 @@ struct Cfg {
     static constexpr uint32_t kAccCols = kNA * BN;                // one accumulator set
     static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
     static constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
-    // one TMEM buffer at BN=256: its epilogue stalls the MMA, so it gets 16 warps
+    // one TMEM buffer at BN=256: its epilogue stalls the MMA, so it gets 16
+    // warps (8 beside the e4m3 converters, within the threads' register room)
     static constexpr int kEpiWarps = BN >= 256 ? (W8 ? 8 : 16) : 4;
     static constexpr int kConvWarps = W8 ? kConvThreads / 32 : 0;
     static constexpr int kConvFirstWarp = 2 + kEpiWarps;

@@ -93,6 +93,10 @@ def test_profiled_traffic_scaling_and_staleness(tmp_path, monkeypatch):
     assert bench.profiled_traffic("small", 1000.0) == 1100
     assert bench.profiled_traffic("full", 5000.0) == 5500
     assert bench.profiled_traffic("absent", 5000.0) is None
+    # an edit of the comments keeps the capture; an edit of the code voids it
+    (tmp_path / "split_weight_b200" / "csrc" / "k.cuh").write_text(
+        "// a note\nkernel  /* block\n comment */ v1 // trailing\n")
+    assert bench.profiled_traffic("full", 5000.0) == 5500
     (tmp_path / "split_weight_b200" / "csrc" / "k.cuh").write_text("kernel v2")
     assert bench.profiled_traffic("full", 5000.0) is None
 
