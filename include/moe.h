@@ -377,7 +377,9 @@ MOE_API moe_status moe_combine(int32_t T, int32_t k, int32_t H, const void *y_pe
  * Remote-expert prefetch into the alternate buffer (explainer, prefetch
  * figure: while a rank computes layer l, the copy engine fetches layer l+1's
  * remote experts into the alternate buffer; fetch-path figure: the pull is a
- * cudaMemcpyAsync on the copy engine, not on the SMs).
+ * cudaMemcpyAsync on the copy engine, not on the SMs).  Between two buffers
+ * of one GPU the driver runs the copy as a kernel on the SMs (measured on
+ * B200), so there the fetch competes with the compute for the SMs.
  *
  * Enqueues on copy_stream: a wait on wait_free (if not NULL: the event the
  * compute stream recorded after the last use of dst), the copy of `bytes`
